@@ -1,0 +1,6 @@
+"""fp64 CPU oracle for exact attention -- test infrastructure only.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+legs import this package.  The CUDA path never does.
+"""
+from .attention import attention_ref, attention_ref_rows, attention_probs  # noqa: F401

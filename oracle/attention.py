@@ -1,0 +1,164 @@
+"""Plain fp64 CPU oracle for exact softmax attention (forward) and its logsumexp.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may call it.  It shares no code,
+header, table or helper with the CUDA path.
+
+What it computes (the plain definition, written out):
+
+    s_ij   = scale * sum_k q_ik k_jk                  for j in allowed(i)
+    LSE_i  = log sum_{j in allowed(i)} exp(s_ij)
+    P_ij   = exp(s_ij - LSE_i)
+    O_i    = sum_j P_ij v_j
+    allowed(i) = {0..N-1}  (non-causal)   or   {0..i}  (causal)
+
+Sources (web pages about Tri Dao, "FlashAttention-2: Faster Attention with
+Better Parallelism and Work Partitioning", arXiv 2307.08691):
+
+* arXiv abstract page, "Abstract": the method computes attention "with no
+  approximation"; the standard layer's runtime and memory are quadratic in the
+  sequence length because it forms the full score matrix.
+* iplexlaw blog "FlashAttention-2: making long-context attention run
+  efficiently on GPUs", section "Why long inputs put pressure on memory": a
+  conventional implementation materialises the score and probability
+  matrices -- which is exactly what this oracle does, on purpose.
+* same blog, section "Tiling preserves the attention calculation": the tiled
+  method reaches the globally normalised softmax result (only floating-point
+  rounding differs), so this untiled definition is the result it must match.
+* same blog, section "Three changes improve GPU utilisation": causal masking
+  (keys after the query are excluded).
+
+Readings where the pages are silent (each is also listed in the design notes):
+
+* scale is the caller's; the benchmark uses 1/sqrt(d).
+* causal alignment: query and key sequences have the same length N, so the
+  mask is "key index j > query index i is excluded"; every row keeps >= 1 key.
+* LSE is the natural log of sum exp(scaled scores), i.e. after scale.
+* an empty row (no allowed key; unreachable with N_q == N_k) gives O = 0 and
+  LSE = -inf.
+
+The oracle is NOT tiled over keys and uses no online softmax: per (b, h) it
+materialises S for a block of query rows (at most ``row_block`` rows at a time
+so N = 16k fits in RAM; row blocking does not change any value, each row is
+computed from all of its keys at once), subtracts the row max, exponentiates,
+normalises, and multiplies by V.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = ["attention_ref", "attention_ref_rows", "attention_probs"]
+
+
+def _as_f64(x) -> np.ndarray:
+    a = np.asarray(x, dtype=np.float64)
+    if a.ndim != 4:
+        raise ValueError(f"expected a [B,H,N,d] array, got shape {a.shape}")
+    return a
+
+
+def _allowed_mask(rows: np.ndarray, n_keys: int, causal: bool) -> np.ndarray:
+    """Boolean [len(rows), n_keys]: True where key j is allowed for query row i.
+
+    Causal masking excludes keys after the query (iplexlaw blog, "Three changes
+    improve GPU utilisation" names causal-mask handling); with equal query and
+    key lengths that is j > i.
+    """
+    j = np.arange(n_keys)[None, :]
+    if causal:
+        return j <= rows[:, None]
+    return np.ones((rows.shape[0], n_keys), dtype=bool)
+
+
+def _rows_one_head(q_rows: np.ndarray, k: np.ndarray, v: np.ndarray,
+                   rows: np.ndarray, causal: bool, scale: float):
+    """Exact attention for selected query rows of one (batch, head).
+
+    q_rows: [R, d] (the query vectors of ``rows``), k, v: [N, d].
+    Returns (O [R, d], LSE [R]) in float64.
+    """
+    n_keys = k.shape[0]
+    # Scores: the full R x N block, materialised (the "standard attention"
+    # the abstract contrasts with the tiled method).
+    s = scale * (q_rows @ k.T)
+    allowed = _allowed_mask(rows, n_keys, causal)
+    s = np.where(allowed, s, -np.inf)
+    m = np.max(s, axis=1, keepdims=True)                 # row max over allowed keys
+    empty = ~np.isfinite(m)                              # row with no allowed key
+    m_safe = np.where(empty, 0.0, m)
+    e = np.exp(s - m_safe)                               # exp(-inf) = 0 on masked keys
+    l = np.sum(e, axis=1, keepdims=True)                 # row sum
+    with np.errstate(divide="ignore", invalid="ignore"):
+        p = np.where(empty, 0.0, e / np.where(empty, 1.0, l))
+        lse = np.where(empty[:, 0], -np.inf, m_safe[:, 0] + np.log(np.where(empty[:, 0], 1.0, l[:, 0])))
+    o = p @ v
+    return o, lse
+
+
+def attention_ref(q, k, v, causal: bool = False, scale: float | None = None,
+                  row_block: int = 2048):
+    """Exact attention forward for [B, H, N, d] inputs.
+
+    Returns ``(O, LSE)``: O float64 [B, H, N, d], LSE float64 [B, H, N]
+    (natural log).  Inputs of any real dtype are upcast to float64 first, so
+    bf16 values are taken exactly.
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, H, N, d = q.shape
+    if k.shape != (B, H, N, d) or v.shape != (B, H, N, d):
+        raise ValueError("q, k, v must share the shape [B, H, N, d]")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.empty((B, H, N, d), dtype=np.float64)
+    lse = np.empty((B, H, N), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            for r0 in range(0, N, row_block):
+                rows = np.arange(r0, min(N, r0 + row_block))
+                ob, lb = _rows_one_head(q[b, h, rows], k[b, h], v[b, h], rows,
+                                        causal, float(scale))
+                o[b, h, rows] = ob
+                lse[b, h, rows] = lb
+    return o, lse
+
+
+def attention_ref_rows(q, k, v, b: int, h: int, rows, causal: bool = False,
+                       scale: float | None = None):
+    """Exact attention for a sample of query rows of one head.
+
+    Same definition as :func:`attention_ref`, evaluated only for ``rows`` of
+    head (b, h); used to check full-size launches on sampled outputs.
+    q, k, v may be any array-likes indexable as [B, H, N, d] (e.g. float64
+    numpy views of bf16 tensors).  Returns (O [R, d], LSE [R]) float64.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    qb = np.asarray(q[b, h], dtype=np.float64)
+    kb = np.asarray(k[b, h], dtype=np.float64)
+    vb = np.asarray(v[b, h], dtype=np.float64)
+    d = qb.shape[-1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    return _rows_one_head(qb[rows], kb, vb, rows, causal, float(scale))
+
+
+def attention_probs(q, k, causal: bool = False, scale: float | None = None):
+    """The materialised probability matrix P [B, H, N, N] (small inputs only).
+
+    P_ij = exp(s_ij - LSE_i) on allowed keys, 0 elsewhere.  Exposed so tests
+    can check the row-stochastic property directly.
+    """
+    q, k = _as_f64(q), _as_f64(k)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    p = np.zeros((B, H, N, N), dtype=np.float64)
+    rows = np.arange(N)
+    allowed = _allowed_mask(rows, N, causal)
+    for b in range(B):
+        for h in range(H):
+            s = np.where(allowed, float(scale) * (q[b, h] @ k[b, h].T), -np.inf)
+            m = np.max(s, axis=1, keepdims=True)
+            e = np.exp(s - m)
+            p[b, h] = e / np.sum(e, axis=1, keepdims=True)
+    return p
