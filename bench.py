@@ -1,0 +1,363 @@
+#!/usr/bin/env python3
+"""Benchmark of the B200 exact-attention forward (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fa2|reference] [--workload NAME]
+
+A step is one call of the forward over the whole workload (one kernel launch).
+The default workload is B=8, H=16, N=2048, d=128, causal, bf16 Q/K/V drawn
+i.i.d. N(0,1) from seed 0, scale 1/sqrt(128) (16k tokens, hidden 2048).  The
+metric is forward TFLOP/s with FLOP = 4*B*H*N^2*d, halved when causal.
+
+N > 1 (launched with torch.distributed.run): every rank runs the same
+workload on its own GPU, i.e. its own shard of N x B sequences; the heads are
+independent, so there is no collective on the data path (weak scaling).  The
+value is the FLOPs of all ranks divided by the slowest rank's time.
+
+``--impl reference`` times the fp64 CPU oracle on this host's cores instead,
+each step on a bounded sample of heads of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attn fwd TFLOP/s (bf16, N=512–16k, d=64/128) and % of B200 dense BF16 peak"
+DEFAULT_WORKLOAD = "B8_H16_N2048_d128_causal"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_BF16_TFLOPS = 2250.0
+KERNEL_SOURCES = ["exact_tiled_attention_45_b200/csrc/fa2_fwd.cu", "exact_tiled_attention_45_b200/csrc/sm100_ptx.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="fa2", choices=["fa2", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the timed oracle sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, src_hash: str):
+    """DRAM bytes per launch from an ncu capture of this exact kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        with open(path) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 3 and not line.startswith("#") and parts[0] == src_hash and parts[1] == workload:
+                    return float(parts[2])
+    except OSError:
+        pass
+    return None
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML (read-only)."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, torch_device):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            try:
+                uuid = str(torch.cuda.get_device_properties(torch_device).uuid)
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(torch_device.index or 0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _sample(self):
+        nv = self._nv
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+            self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(0.005)
+
+    def start(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+            self._sample()
+
+    def summary(self):
+        if self._nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        s = sorted(self.samples)
+        med = s[len(s) // 2] if s else None
+        names = [k for k, bit in self.REASONS.items() if self.reasons & bit and k != "gpu_idle"]
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(s)}
+
+
+def cpu_oracle_sample(w, budget_s: float, q, k, v):
+    """Time the fp64 oracle on whole heads of the workload until the budget is spent."""
+    import numpy as np
+    import torch
+    from oracle import attention_ref
+    cores = torch.get_num_threads()
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    done, flops, t0 = 0, 0.0, time.perf_counter()
+    per_head = w.flops / (w.B * w.H)
+    for b, h in heads:
+        attention_ref(q[b:b + 1, h:h + 1].double().numpy(), k[b:b + 1, h:h + 1].double().numpy(),
+                      v[b:b + 1, h:h + 1].double().numpy(), causal=w.causal, scale=w.d ** -0.5)
+        done += 1
+        flops += per_head
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": int(cores), "kind": "oracle",
+            "sample": f"{done} of {len(heads)} heads of {w.name} (fp64 NumPy, {dt:.1f} s)",
+            "seconds": round(dt, 2)}, np
+
+
+def run_reference(args, w):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import torch
+    from exact_tiled_attention_45_b200.inputs import make_qkv
+    from oracle import attention_ref
+    heads_per_step = 1
+    q, k, v = make_qkv(w.B, w.H, w.N, w.d, seed=0, qk_mult=w.qk_mult)
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    per_head = w.flops / (w.B * w.H)
+
+    def step(i):
+        for t in range(heads_per_step):
+            b, h = heads[(i * heads_per_step + t) % len(heads)]
+            attention_ref(q[b:b + 1, h:h + 1].double().numpy(), k[b:b + 1, h:h + 1].double().numpy(),
+                          v[b:b + 1, h:h + 1].double().numpy(), causal=w.causal, scale=w.d ** -0.5)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = per_head * heads_per_step * args.steps / dt / 1e12
+    cores = torch.get_num_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(w.as_dict(), sample=f"{heads_per_step} head(s) of {w.B * w.H} per step"),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": int(cores), "kind": "oracle",
+                         "sample": f"{heads_per_step} head(s) per step of {w.name}, fp64 NumPy on host cores"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    from exact_tiled_attention_45_b200.inputs import WORKLOADS
+    if args.workload not in WORKLOADS:
+        raise SystemExit(f"unknown workload {args.workload}; choose from {sorted(WORKLOADS)}")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    import exact_tiled_attention_45_b200 as fa2
+    from exact_tiled_attention_45_b200.inputs import make_qkv
+
+    world, rank, local = dist_env()
+    if args.steps < 1 or args.warmup < 3:
+        raise SystemExit("need --steps >= 1 and --warmup >= 3")
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+
+    # Each rank draws its own shard of sequences (seed = rank) and keeps it resident.
+    q_h, k_h, v_h = make_qkv(w.B, w.H, w.N, w.d, seed=rank, qk_mult=w.qk_mult)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    in_bytes = 3 * q.numel() * 2
+    out_bytes = o.numel() * 2 + lse.numel() * 4
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = None
+    if in_bytes <= l2_bytes:
+        flush = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev)
+
+    def step():
+        if flush is not None:
+            flush.zero_()
+        fa2.fwd(q, k, v, causal=w.causal, out=o, lse=lse, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    fa2.sync_status(stream)
+
+    sampler = ClockSampler(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    if flush is None:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        total_ms = ev0.elapsed_time(ev1)
+        kernel_ms = total_ms / args.steps
+    else:
+        # L2 is flushed before every step; only the kernels are timed.
+        kernel_ms_sum = 0.0
+        for _ in range(args.steps):
+            flush.zero_()
+            ev0.record(stream)
+            fa2.fwd(q, k, v, causal=w.causal, out=o, lse=lse, stream=stream)
+            ev1.record(stream)
+            ev1.synchronize()
+            kernel_ms_sum += ev0.elapsed_time(ev1)
+        total_ms = kernel_ms_sum
+        kernel_ms = kernel_ms_sum / args.steps
+    sampler.stop()
+    barrier()
+    fa2.sync_status(stream)
+
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    ms_per_step = max_ms / args.steps
+    total_flops = w.flops * world
+    value = total_flops / (ms_per_step * 1e-3) / 1e12
+
+    # End to end through the host-buffer entry point: pinned host inputs in,
+    # host outputs back, copies inside the timed region.
+    e2e = None
+    if not args.no_e2e:
+        qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+        op = torch.empty_like(qp).pin_memory()
+        lp = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+        ws = torch.empty(fa2.workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+        e2e_steps = max(3, min(args.steps, 10))
+        for _ in range(2):
+            fa2.fwd_host(qp, kp, vp, causal=w.causal, out=op, lse=lp, workspace=ws, stream=stream)
+        barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for _ in range(e2e_steps):
+            fa2.fwd_host(qp, kp, vp, causal=w.causal, out=op, lse=lp, workspace=ws, stream=stream)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        te = torch.tensor([ev0.elapsed_time(ev1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te.item()) / e2e_steps
+        e2e = {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes, "steps": e2e_steps}
+        del qp, kp, vp, op, lp, ws
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    achieved = w.flops / (kernel_ms * 1e-3) / 1e12
+    src = source_hash()
+    traffic = recorded_traffic(w.name, src)
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu, _ = cpu_oracle_sample(w, args.cpu_seconds, q_h, k_h, v_h)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(w.as_dict(), seed="rank", scale=f"1/sqrt({w.d})",
+                       l2=("inputs larger than L2" if flush is None else "L2 flushed before every step"),
+                       parallelism=("single GPU" if world == 1 else f"{world} ranks, independent heads, no collective")),
+        "pct_of_peak": {"measured_burst": 100.0 * achieved / peak, "measured_sustained": 100.0 * achieved / peak_sus,
+                        "spec_2250": 100.0 * achieved / SPEC_BF16_TFLOPS, "peaks": peak_kind},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_kind} bf16 burst",
+                     "kernel": "fa2_fwd_kernel", "src": src},
+        "clocks": sampler.summary(),
+        "gpu_launches": args.steps,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,169 @@
+"""Python binding of the C ABI in ``include/fa2.h`` (ctypes; marshalling only).
+
+Every step of the attention forward runs in the CUDA kernels of libfa2.so;
+this module only checks tensor properties, allocates outputs with torch and
+passes raw pointers and the current stream.  There is no fallback: if the
+library is missing or a call fails, a RuntimeError is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libfa2.so")
+
+FA2_OK, FA2_ERR_INVALID_ARG, FA2_ERR_UNSUPPORTED, FA2_ERR_CUDA, FA2_ERR_TIMEOUT = range(5)
+
+#: Every symbol the header declares.
+EXPORTS = ("fa2_fwd", "fa2_fwd_host", "fa2_fwd_host_workspace_bytes", "fa2_sync_status",
+           "fa2_fwd_inject_timeout", "fa2_strerror", "fa2_last_error_detail", "fa2_version")
+
+_lib = None
+
+_vp, _int, _float = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+_FWD_ARGS = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _float]
+
+
+def load() -> ctypes.CDLL:
+    """Load libfa2.so (built in-tree); raise if it is not there."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m exact_tiled_attention_45_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    lib.fa2_fwd.argtypes = _FWD_ARGS + [_vp]
+    lib.fa2_fwd.restype = _int
+    lib.fa2_fwd_host.argtypes = _FWD_ARGS + [_vp, ctypes.c_size_t, _vp]
+    lib.fa2_fwd_host.restype = _int
+    lib.fa2_fwd_host_workspace_bytes.argtypes = [_int, _int, _int, _int]
+    lib.fa2_fwd_host_workspace_bytes.restype = ctypes.c_size_t
+    lib.fa2_sync_status.argtypes = [_vp]
+    lib.fa2_sync_status.restype = _int
+    lib.fa2_fwd_inject_timeout.argtypes = _FWD_ARGS + [ctypes.c_ulonglong, _vp]
+    lib.fa2_fwd_inject_timeout.restype = _int
+    lib.fa2_strerror.argtypes = [_int]
+    lib.fa2_strerror.restype = ctypes.c_char_p
+    lib.fa2_last_error_detail.argtypes = []
+    lib.fa2_last_error_detail.restype = ctypes.c_char_p
+    lib.fa2_version.argtypes = []
+    lib.fa2_version.restype = _int
+    _lib = lib
+    return lib
+
+
+class FA2Error(RuntimeError):
+    def __init__(self, status: int, lib):
+        self.status = status
+        msg = lib.fa2_strerror(status).decode()
+        detail = lib.fa2_last_error_detail().decode()
+        super().__init__(f"fa2 status {status} ({msg}){': ' + detail if detail else ''}")
+
+
+def _check(status: int, lib) -> None:
+    if status != FA2_OK:
+        raise FA2Error(status, lib)
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _check_qkv(q, k, v, device: str):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be [B, H, N, d], got {tuple(t.shape)}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.device.type != device:
+            raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must share the shape [B, H, N, d]")
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, scale: float | None = None,
+        out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
+    """Exact attention forward on CUDA tensors.  Returns (O bf16, LSE fp32).
+
+    Asynchronous on ``stream`` (default: torch's current stream).
+    """
+    lib = load()
+    _check_qkv(q, k, v, "cuda")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    st = lib.fa2_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                     B, H, N, d, int(bool(causal)), float(scale), _stream_handle(stream))
+    _check(st, lib)
+    return out, lse
+
+
+def sync_status(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel reported a timed-out wait."""
+    lib = load()
+    _check(lib.fa2_sync_status(_stream_handle(stream)), lib)
+
+
+def workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(load().fa2_fwd_host_workspace_bytes(B, H, N, d))
+
+
+def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, scale: float | None = None,
+             out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+             workspace: torch.Tensor | None = None, stream=None):
+    """End-to-end call on HOST tensors (pinned for full copy bandwidth).
+
+    Copies q, k, v to the device, runs the kernel, copies O and LSE back and
+    returns after they have landed.  ``workspace`` is an optional uint8 CUDA
+    tensor of at least :func:`workspace_bytes` bytes, reused across calls.
+    """
+    lib = load()
+    _check_qkv(q, k, v, "cpu")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
+    if workspace.numel() < need:
+        raise ValueError(f"workspace needs {need} bytes")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32)
+    st = lib.fa2_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                          B, H, N, d, int(bool(causal)), float(scale), workspace.data_ptr(),
+                          workspace.numel(), _stream_handle(stream))
+    _check(st, lib)
+    return out, lse
+
+
+def fwd_inject_timeout(q, k, v, causal=False, scale=None, timeout_ns: int = 50_000_000, stream=None):
+    """Failure-path test hook: run the kernel with the Q-tile load withheld.
+
+    Returns the status of :func:`sync_status` (expected FA2_ERR_TIMEOUT).
+    """
+    lib = load()
+    _check_qkv(q, k, v, "cuda")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    h = _stream_handle(stream)
+    st = lib.fa2_fwd_inject_timeout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                    B, H, N, d, int(bool(causal)), float(scale), int(timeout_ns), h)
+    _check(st, lib)
+    return lib.fa2_sync_status(h)

@@ -1,0 +1,666 @@
+// Exact attention forward for B200 (sm_100a): tiled, online softmax, tcgen05
+// tensor-core MMAs accumulating in tensor memory, TMA tile loads, and
+// warp-specialised roles.
+//
+// Method (FlashAttention-2, Tri Dao, arXiv 2307.08691):
+//  * arXiv abstract page, "Abstract" (1)-(3) and iplexlaw blog "FlashAttention-2:
+//    making long-context attention run efficiently on GPUs", section "Three
+//    changes improve GPU utilisation":
+//      (1) fewer non-matmul FLOPs: the running max/sum live in registers, the
+//          1/l normalisation is deferred to the epilogue, exponentials use exp2
+//          with the softmax scale folded into one FMA, and only the diagonal
+//          (causal) or ragged tail tile is masked element by element;
+//      (2) parallel over the sequence: one CTA per (query tile, head, batch);
+//      (3) work split without shared-memory reductions: each softmax thread
+//          owns one query row (one TMEM lane) from scores to output.
+//  * iplexlaw blog, section "Tiling preserves the attention calculation":
+//    K/V are streamed through on-chip memory tile by tile; the online softmax
+//    rescales partial outputs so the result is the globally normalised one.
+//
+// B200 design (not in the pages, which describe A100 kernels):
+//  * warp 4 = TMA producer (Q once; K and V through separate rings);
+//  * warp 5 = MMA issuer: S_j = Q K_j^T (SS form) into one of two TMEM score
+//    buffers, O += P_j V_j (TS form: P read from TMEM), commits to mbarriers;
+//  * warps 0-3 = softmax / correction / epilogue, thread t <-> query row t
+//    <-> TMEM lane t;
+//  * the O rescale is skipped unless a row's running max grows by more than
+//    RESCALE_THRESHOLD (log2 units).  The stale max is used consistently for
+//    P, the running sum and the final LSE, so the result is unchanged (the
+//    exponentials stay below 2^RESCALE_THRESHOLD).
+//  * every wait is bounded; on time-out the kernel records a status word,
+//    drains its own in-flight copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include "fa2.h"
+#include "sm100_ptx.cuh"
+
+namespace fa2 {
+
+using namespace ptx;
+
+constexpr int BM = 128;  // query rows per CTA (one tcgen05 M=128 tile)
+constexpr int BN = 128;  // keys per K/V tile
+constexpr int NUM_THREADS = 192;
+constexpr int PRODUCER_WARP = 4;
+constexpr int MMA_WARP = 5;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_S0 = 0;    // score buffer 0: 128 fp32 columns
+constexpr uint32_t TM_S1 = 128;  // score buffer 1
+constexpr uint32_t TM_P = 256;   // probabilities: 128 bf16 per row = 64 columns
+constexpr uint32_t TM_O = 384;   // output accumulator: d fp32 columns
+constexpr float RESCALE_THRESHOLD = 8.0f;
+
+// Device status word: bit 0 = a bounded wait gave up; bits 8..11 = role.
+__device__ unsigned int g_fa2_status = 0;
+constexpr unsigned int STATUS_TIMEOUT = 1u;
+constexpr unsigned int ROLE_PRODUCER = 1u << 8, ROLE_MMA = 2u << 8, ROLE_SOFTMAX = 3u << 8,
+                       ROLE_DRAIN = 4u << 8;
+
+template <int HD>
+struct Cfg {
+  static_assert(HD == 64 || HD == 128, "head dimension");
+  static constexpr int KCH = HD / 64;                  // 64-element (128-byte) column chunks
+  static constexpr int CHUNK_BYTES = 128 * 128;        // 128 rows x 128 bytes
+  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;  // one 128-row Q/K/V tile
+  static constexpr int KS = (HD == 128) ? 2 : 3;       // K ring stages
+  static constexpr int VS = (HD == 128) ? 2 : 3;       // V ring stages
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VS * TILE_BYTES;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct Params {
+  __nv_bfloat16* o;
+  float* lse;
+  int N;
+  int H;
+  int n_q_tiles;
+  int n_kv_tiles;
+  float scale_log2;  // scale * log2(e)
+  unsigned long long timeout_ns;
+  int inject_timeout;  // test hook: withhold the Q load
+};
+
+struct Barriers {
+  uint64_t q_full;
+  uint64_t k_full[3], k_empty[3];
+  uint64_t v_full[3], v_empty[3];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full;
+  uint64_t pv_done;
+  uint64_t mma_final;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Bounded wait.  Returns false (and records the time-out once) if the phase
+// did not complete within timeout_ns, or if another role already gave up.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                             unsigned long long timeout_ns, unsigned int role) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      *abort_flag = 1;
+      atomicOr(&g_fa2_status, STATUS_TIMEOUT | role);
+      return false;
+    }
+  }
+}
+
+// Bounded wait used while draining: ignores the abort flag.
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, unsigned long long timeout_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      atomicOr(&g_fa2_status, STATUS_TIMEOUT | ROLE_DRAIN);
+      return false;
+    }
+  }
+  return true;
+}
+
+template <int HD, bool CAUSAL>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  using C = Cfg<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte-swizzle atoms.
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + C::OFF_BAR);
+  volatile int* abort_flag = &bars->abort;
+
+  const uint32_t sQ = base + C::OFF_Q;
+  const uint32_t sK = base + C::OFF_K;
+  const uint32_t sV = base + C::OFF_V;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int qt = CAUSAL ? (p.n_q_tiles - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+  const int bh = static_cast<int>(blockIdx.z) * p.H + static_cast<int>(blockIdx.y);
+  const int q0 = qt * BM;
+  const int nkv = CAUSAL ? min(qt + 1, p.n_kv_tiles) : p.n_kv_tiles;
+
+  const uint32_t b_q_full = smem_u32(&bars->q_full);
+  const uint32_t b_pfull = smem_u32(&bars->p_full);
+  const uint32_t b_pvdone = smem_u32(&bars->pv_done);
+  const uint32_t b_final = smem_u32(&bars->mma_final);
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_q_full, 1);
+    for (int s = 0; s < C::KS; ++s) {
+      mbar_init(smem_u32(&bars->k_full[s]), 1);
+      mbar_init(smem_u32(&bars->k_empty[s]), 1);
+    }
+    for (int s = 0; s < C::VS; ++s) {
+      mbar_init(smem_u32(&bars->v_full[s]), 1);
+      mbar_init(smem_u32(&bars->v_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&bars->s_full[s]), 1);
+      mbar_init(smem_u32(&bars->s_free[s]), 4);
+    }
+    mbar_init(b_pfull, 4);
+    mbar_init(b_pvdone, 1);
+    mbar_init(b_final, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(smem_u32(&bars->tmem_base), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == PRODUCER_WARP && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == PRODUCER_WARP) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const bool load_q = !p.inject_timeout;
+      if (load_q) {
+        mbar_arrive_expect_tx(b_q_full, C::TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * C::CHUNK_BYTES, &tm_q, b_q_full, c * 64, q0, bh);
+      }
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < nkv; ++j) {
+        const int ks = j % C::KS;
+        if (j >= C::KS &&
+            !wait_bounded(smem_u32(&bars->k_empty[ks]), ((j / C::KS) - 1) & 1, abort_flag, p.timeout_ns,
+                          ROLE_PRODUCER))
+          break;
+        const uint32_t kb = smem_u32(&bars->k_full[ks]);
+        mbar_arrive_expect_tx(kb, C::TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sK + ks * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_k, kb, c * 64, j * BN, bh);
+        ++k_issued;
+        const int vs = j % C::VS;
+        if (j >= C::VS &&
+            !wait_bounded(smem_u32(&bars->v_empty[vs]), ((j / C::VS) - 1) & 1, abort_flag, p.timeout_ns,
+                          ROLE_PRODUCER))
+          break;
+        const uint32_t vb = smem_u32(&bars->v_full[vs]);
+        mbar_arrive_expect_tx(vb, C::TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sV + vs * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_v, vb, c * 64, j * BN, bh);
+        ++v_issued;
+      }
+      // Drain: every load this thread issued must land before the CTA exits.
+      if (load_q) wait_drain(b_q_full, 0, p.timeout_ns);
+      for (int t = (k_issued > C::KS ? k_issued - C::KS : 0); t < k_issued; ++t)
+        wait_drain(smem_u32(&bars->k_full[t % C::KS]), (t / C::KS) & 1, p.timeout_ns);
+      for (int t = (v_issued > C::VS ? v_issued - C::VS : 0); t < v_issued; ++t)
+        wait_drain(smem_u32(&bars->v_full[t % C::VS]), (t / C::VS) & 1, p.timeout_ns);
+    }
+  } else if (warp == MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
+      bool ok = wait_bounded(b_q_full, 0, abort_flag, p.timeout_ns, ROLE_MMA);
+      for (int j = 0; ok && j <= nkv; ++j) {
+        if (j < nkv) {
+          const int ks = j % C::KS;
+          const int sb = j & 1;
+          if (!wait_bounded(smem_u32(&bars->k_full[ks]), (j / C::KS) & 1, abort_flag, p.timeout_ns, ROLE_MMA))
+            break;
+          if (j >= 2 &&
+              !wait_bounded(smem_u32(&bars->s_free[sb]), ((j - 2) >> 1) & 1, abort_flag, p.timeout_ns, ROLE_MMA))
+            break;
+          tc_fence_after();
+          const uint32_t d_s = tmem + (sb ? TM_S1 : TM_S0);
+          const uint32_t kbase = sK + ks * C::TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+            mma_ss(d_s, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024), IDESC_S,
+                   kk > 0 ? 1u : 0u);
+          }
+          mma_commit(smem_u32(&bars->s_full[sb]));
+          mma_commit(smem_u32(&bars->k_empty[ks]));
+        }
+        if (j >= 1) {
+          const int i = j - 1;
+          const int vs = i % C::VS;
+          if (!wait_bounded(b_pfull, i & 1, abort_flag, p.timeout_ns, ROLE_MMA)) break;
+          if (!wait_bounded(smem_u32(&bars->v_full[vs]), (i / C::VS) & 1, abort_flag, p.timeout_ns, ROLE_MMA))
+            break;
+          tc_fence_after();
+          const uint32_t vbase = sV + vs * C::TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            mma_ts(tmem + TM_O, tmem + TM_P + kk * 8, smem_desc_sw128(vbase + kk * 2048, C::CHUNK_BYTES, 1024),
+                   IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(smem_u32(&bars->v_empty[vs]));
+          mma_commit(b_pvdone);
+        }
+      }
+      // Drain: all MMAs issued by this thread complete before TMEM is freed.
+      mma_commit(b_final);
+      wait_drain(b_final, 0, p.timeout_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps 0..3
+    const int r = threadIdx.x;  // query row within the tile == TMEM lane
+    const int row_g = q0 + r;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float c_log2 = p.scale_log2;
+    float m = -INFINITY;  // running max of scale*log2(e)*s (possibly stale, see header)
+    float l = 0.f;        // running sum of exp2(...) relative to m
+    bool ok = true;
+    for (int i = 0; i < nkv; ++i) {
+      const int sb = i & 1;
+      ok = wait_bounded(smem_u32(&bars->s_full[sb]), (i >> 1) & 1, abort_flag, p.timeout_ns, ROLE_SOFTMAX);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[4][32];
+      const uint32_t s_addr = lane_addr + (sb ? TM_S1 : TM_S0);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, s[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence32(s[c]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[sb]));
+
+      const int kv0 = i * BN;
+      const bool diag = CAUSAL && (kv0 + BN > q0);       // tile reaches past this CTA's first row
+      const bool tail = !CAUSAL && (kv0 + BN > p.N);     // ragged last key tile
+      if (diag || tail) {
+        const int lim = diag ? (row_g - kv0) : (p.N - 1 - kv0);  // last allowed column
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e > lim) s[c][e] = __float_as_uint(-INFINITY);
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(s[c][e]));
+      const float m_cand = mx * c_log2;
+      float m_new = m;
+      if (m_cand > m + RESCALE_THRESHOLD) m_new = m_cand;  // also taken on the first tile (m = -inf)
+      const bool rescale = (i > 0) && (m_new != m);
+      const float alpha = rescale ? ex2(m - m_new) : 1.f;
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+
+      float rowsum = 0.f;
+      uint32_t pk[2][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float p0 = ex2(fmaf(__uint_as_float(s[c][e]), c_log2, -m_use));
+          const float p1 = ex2(fmaf(__uint_as_float(s[c][e + 1]), c_log2, -m_use));
+          rowsum += p0 + p1;
+          pk[c >> 1][(c & 1) * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
+        }
+      }
+      if (i > 0) {
+        // O and the P buffer are in use by PV_{i-1} until it completes.
+        ok = wait_bounded(b_pvdone, (i - 1) & 1, abort_flag, p.timeout_ns, ROLE_SOFTMAX);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < HD / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + TM_O + c * 32, o);
+            tmem_wait_ld();
+            reg_fence32(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(lane_addr + TM_O + c * 32, o);
+          }
+        }
+      }
+      tmem_st32(lane_addr + TM_P, pk[0]);
+      tmem_st32(lane_addr + TM_P + 32, pk[1]);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_pfull);
+      l = l * alpha + rowsum;
+      m = m_new;
+    }
+    if (ok && nkv > 0) {
+      ok = wait_bounded(b_pvdone, (nkv - 1) & 1, abort_flag, p.timeout_ns, ROLE_SOFTMAX);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const bool store = row_g < p.N;
+      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (store ? row_g : 0)) * HD;
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(lane_addr + TM_O + c * 32, o);
+        tmem_wait_ld();
+        reg_fence32(o);
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        }
+      }
+      if (store) {
+        const float lse = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        p.lse[static_cast<size_t>(bh) * p.N + row_g] = lse;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ====================================================================== host
+
+static thread_local char g_detail[512] = "";
+
+static void set_detail(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn) return fn;
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  return fn;
+}
+
+// View a [B*H, N, d] bf16 tensor as a 3-D TMA map with 64 x 128 x 1 boxes,
+// 128-byte swizzle.  Rows past N read as zero.
+static int make_tmap(CUtensorMap* tm, const void* ptr, int d, int N, int BH) {
+  auto enc = get_encode_fn();
+  if (!enc) {
+    set_detail("cuTensorMapEncodeTiled entry point unavailable");
+    return FA2_ERR_CUDA;
+  }
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_detail("cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+    return FA2_ERR_CUDA;
+  }
+  return FA2_OK;
+}
+
+static bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+static int validate(const void* q, const void* k, const void* v, const void* o, const float* lse, int B, int H,
+                    int N, int d, float scale) {
+  if (!q || !k || !v || !o || !lse) {
+    set_detail("null pointer");
+    return FA2_ERR_INVALID_ARG;
+  }
+  if (B < 1 || H < 1 || N < 1 || B > 65535 || H > 65535) {
+    set_detail("bad sizes B=%d H=%d N=%d", B, H, N);
+    return FA2_ERR_INVALID_ARG;
+  }
+  if (!std::isfinite(scale)) {
+    set_detail("scale is not finite");
+    return FA2_ERR_INVALID_ARG;
+  }
+  if (d != 64 && d != 128) {
+    set_detail("head dimension %d not supported (64 or 128)", d);
+    return FA2_ERR_UNSUPPORTED;
+  }
+  const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                        reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o);
+  if ((mis & 15u) || (reinterpret_cast<uintptr_t>(lse) & 3u)) {
+    set_detail("misaligned pointer (q/k/v/o need 16 bytes, lse 4)");
+    return FA2_ERR_INVALID_ARG;
+  }
+  const size_t n_elem = static_cast<size_t>(B) * H * N * d;
+  const size_t t_bytes = n_elem * 2, l_bytes = static_cast<size_t>(B) * H * N * 4;
+  if (overlap(o, t_bytes, q, t_bytes) || overlap(o, t_bytes, k, t_bytes) || overlap(o, t_bytes, v, t_bytes) ||
+      overlap(o, t_bytes, lse, l_bytes) || overlap(lse, l_bytes, q, t_bytes) ||
+      overlap(lse, l_bytes, k, t_bytes) || overlap(lse, l_bytes, v, t_bytes)) {
+    set_detail("output buffers overlap inputs or each other");
+    return FA2_ERR_INVALID_ARG;
+  }
+  return FA2_OK;
+}
+
+template <int HD, bool CAUSAL>
+static int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const Params& prm,
+                    int B, int H, cudaStream_t stream) {
+  using C = Cfg<HD>;
+  auto kern = fa2_fwd_kernel<HD, CAUSAL>;
+  static int attr_done_mask = 0;  // per device bit (devices 0..31)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    set_detail("cudaGetDevice failed");
+    return FA2_ERR_CUDA;
+  }
+  if (dev >= 32 || !(attr_done_mask & (1 << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) {
+      set_detail("cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+      return FA2_ERR_CUDA;
+    }
+    if (dev < 32) attr_done_mask |= (1 << dev);
+  }
+  dim3 grid(prm.n_q_tiles, H, B);
+  kern<<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_detail("kernel launch: %s", cudaGetErrorString(e));
+    return FA2_ERR_CUDA;
+  }
+  return FA2_OK;
+}
+
+static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                    int causal, float scale, unsigned long long timeout_ns, int inject, cudaStream_t stream) {
+  g_detail[0] = 0;
+  int st = validate(q, k, v, o, lse, B, H, N, d, scale);
+  if (st != FA2_OK) return st;
+  CUtensorMap tq, tk, tv;
+  const int BH = B * H;
+  if ((st = make_tmap(&tq, q, d, N, BH)) != FA2_OK) return st;
+  if ((st = make_tmap(&tk, k, d, N, BH)) != FA2_OK) return st;
+  if ((st = make_tmap(&tv, v, d, N, BH)) != FA2_OK) return st;
+  Params prm;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.N = N;
+  prm.H = H;
+  prm.n_q_tiles = (N + BM - 1) / BM;
+  prm.n_kv_tiles = (N + BN - 1) / BN;
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+  prm.timeout_ns = timeout_ns;
+  prm.inject_timeout = inject;
+  if (d == 64)
+    return causal ? launch_t<64, true>(tq, tk, tv, prm, B, H, stream)
+                  : launch_t<64, false>(tq, tk, tv, prm, B, H, stream);
+  return causal ? launch_t<128, true>(tq, tk, tv, prm, B, H, stream)
+                : launch_t<128, false>(tq, tk, tv, prm, B, H, stream);
+}
+
+constexpr unsigned long long DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s per wait
+
+}  // namespace fa2
+
+// ====================================================================== C ABI
+extern "C" {
+
+int fa2_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+            int causal, float scale, void* stream) {
+  return fa2::fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, fa2::DEFAULT_TIMEOUT_NS, 0,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int fa2_fwd_inject_timeout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                           int N, int d, int causal, float scale, unsigned long long timeout_ns, void* stream) {
+  if (timeout_ns == 0 || timeout_ns > fa2::DEFAULT_TIMEOUT_NS) {
+    fa2::set_detail("timeout_ns out of range (1 .. 2e9)");
+    return FA2_ERR_INVALID_ARG;
+  }
+  return fa2::fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, timeout_ns, 1,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int fa2_sync_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    fa2::set_detail("cudaStreamSynchronize: %s", cudaGetErrorString(e));
+    return FA2_ERR_CUDA;
+  }
+  unsigned int st = 0;
+  e = cudaMemcpyFromSymbol(&st, fa2::g_fa2_status, sizeof(st));
+  if (e != cudaSuccess) {
+    fa2::set_detail("reading the status word: %s", cudaGetErrorString(e));
+    return FA2_ERR_CUDA;
+  }
+  if (st) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(fa2::g_fa2_status, &zero, sizeof(zero));
+    fa2::set_detail("device status word 0x%x", st);
+    return FA2_ERR_TIMEOUT;
+  }
+  return FA2_OK;
+}
+
+size_t fa2_fwd_host_workspace_bytes(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  const size_t t = ((static_cast<size_t>(B) * H * N * d * 2) + 255) & ~static_cast<size_t>(255);
+  const size_t l = ((static_cast<size_t>(B) * H * N * 4) + 255) & ~static_cast<size_t>(255);
+  return 4 * t + l;
+}
+
+int fa2_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  fa2::g_detail[0] = 0;
+  if (!q || !k || !v || !o || !lse || !workspace) {
+    fa2::set_detail("null pointer");
+    return FA2_ERR_INVALID_ARG;
+  }
+  const size_t need = fa2_fwd_host_workspace_bytes(B, H, N, d);
+  if (need == 0) {
+    if (d != 64 && d != 128 && B >= 1 && H >= 1 && N >= 1) return FA2_ERR_UNSUPPORTED;
+    fa2::set_detail("bad sizes");
+    return FA2_ERR_INVALID_ARG;
+  }
+  if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) {
+    fa2::set_detail("workspace too small or misaligned (need %zu bytes, 256-byte aligned)", need);
+    return FA2_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t tb = static_cast<size_t>(B) * H * N * d * 2;
+  const size_t t = (tb + 255) & ~static_cast<size_t>(255);
+  const size_t lb = static_cast<size_t>(B) * H * N * 4;
+  char* ws = static_cast<char*>(workspace);
+  void *dq = ws, *dk = ws + t, *dv = ws + 2 * t, *dout = ws + 3 * t;
+  float* dl = reinterpret_cast<float*>(ws + 4 * t);
+  cudaError_t e;
+  if ((e = cudaMemcpyAsync(dq, q, tb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dk, k, tb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dv, v, tb, cudaMemcpyHostToDevice, s)) != cudaSuccess) {
+    fa2::set_detail("host-to-device copy: %s", cudaGetErrorString(e));
+    return FA2_ERR_CUDA;
+  }
+  int st = fa2_fwd(dq, dk, dv, dout, dl, B, H, N, d, causal, scale, stream);
+  if (st != FA2_OK) return st;
+  if ((e = cudaMemcpyAsync(o, dout, tb, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(lse, dl, lb, cudaMemcpyDeviceToHost, s)) != cudaSuccess) {
+    fa2::set_detail("device-to-host copy: %s", cudaGetErrorString(e));
+    return FA2_ERR_CUDA;
+  }
+  return fa2_sync_status(stream);
+}
+
+const char* fa2_strerror(int status) {
+  switch (status) {
+    case FA2_OK: return "ok";
+    case FA2_ERR_INVALID_ARG: return "invalid argument";
+    case FA2_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FA2_ERR_CUDA: return "CUDA error";
+    case FA2_ERR_TIMEOUT: return "kernel wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* fa2_last_error_detail(void) { return fa2::g_detail; }
+
+int fa2_version(void) { return 100; }
+
+}  // extern "C"

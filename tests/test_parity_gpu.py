@@ -1,0 +1,170 @@
+"""GPU parity: the sm_100a kernels (through the C ABI) against the fp64 oracle.
+
+Tolerances (bf16 inputs, fp32 accumulation): max |dLSE| <= 1e-3 and
+|dO| <= 1e-2 per element, plus half a bf16 spacing of the exact value: O is
+returned in bf16, and that final rounding alone can reach 2^-5 / 2 = 0.016 for
+|O| in [4, 8), which occurs in the large-logit (x4) workloads.  Small cases
+are compared element by element; full-size workloads on sampled rows that
+include tile boundaries, the first and the last row.
+"""
+import numpy as np
+import pytest
+import torch
+
+from exact_tiled_attention_45_b200 import fwd, fwd_host, sync_status
+from exact_tiled_attention_45_b200.inputs import WORKLOADS, make_qkv
+from oracle import attention_ref, attention_ref_rows
+
+pytestmark = pytest.mark.gpu
+
+O_TOL = 1e-2
+LSE_TOL = 1e-3
+
+
+def bf16_half_spacing(x):
+    a = np.maximum(np.abs(x), 2.0 ** -126)
+    e = np.floor(np.log2(a)).astype(np.int64)
+    return np.ldexp(1.0, e - 8)
+
+
+def assert_close(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
+    o = np.asarray(o_gpu, dtype=np.float64)
+    lse = np.asarray(lse_gpu, dtype=np.float64)
+    assert np.isfinite(o).all() and np.isfinite(lse).all(), f"{what}: non-finite output"
+    err_o = np.abs(o - o_ref)
+    bound = O_TOL + bf16_half_spacing(o_ref)
+    worst = np.unravel_index(np.argmax(err_o - bound), err_o.shape)
+    assert (err_o <= bound).all(), (f"{what}: |dO| {err_o[worst]:.3e} > {bound[worst]:.3e} at {worst} "
+                                    f"(gpu {o[worst]}, ref {o_ref[worst]}); max |dO| {err_o.max():.3e}")
+    err_l = np.abs(lse - lse_ref)
+    assert err_l.max() <= LSE_TOL, f"{what}: max |dLSE| {err_l.max():.3e} at {np.unravel_index(err_l.argmax(), err_l.shape)}"
+    return float(err_o.max()), float(err_l.max())
+
+
+def run_gpu(q, k, v, causal, scale=None):
+    o, lse = fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale)
+    sync_status()
+    return o.double().cpu().numpy(), lse.double().cpu().numpy()
+
+
+SMALL = [
+    # (B, H, N, d, causal, qk_mult)
+    (1, 2, 128, 64, False, 1.0),   # the tiny workload
+    (1, 2, 128, 64, True, 1.0),
+    (2, 3, 384, 64, False, 1.0),
+    (2, 3, 384, 64, True, 1.0),
+    (2, 3, 384, 128, False, 1.0),
+    (2, 3, 384, 128, True, 1.0),
+    (1, 2, 1024, 128, False, 1.0),
+    (1, 2, 1024, 64, True, 1.0),
+    # ragged sequence lengths (last tile partly out of range)
+    (1, 1, 1, 64, False, 1.0),
+    (1, 1, 1, 128, True, 1.0),
+    (1, 1, 7, 128, False, 1.0),
+    (1, 2, 129, 64, False, 1.0),
+    (1, 2, 129, 64, True, 1.0),
+    (1, 2, 320, 128, False, 1.0),
+    (1, 2, 320, 128, True, 1.0),
+    (2, 1, 1000, 64, False, 1.0),
+    (2, 1, 1000, 128, True, 1.0),
+    # large logits (Q, K x4)
+    (2, 2, 512, 128, False, 4.0),
+    (2, 2, 512, 128, True, 4.0),
+    (1, 2, 640, 64, False, 4.0),
+    (1, 2, 640, 64, True, 4.0),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal,mult", SMALL,
+                         ids=[f"B{b}H{h}N{n}d{d}{'c' if c else 'f'}x{int(m)}" for b, h, n, d, c, m in SMALL])
+def test_small_elementwise(B, H, N, d, causal, mult):
+    q, k, v = make_qkv(B, H, N, d, seed=0, qk_mult=mult)
+    o, lse = run_gpu(q, k, v, causal)
+    o_ref, lse_ref = attention_ref(q.double().numpy(), k.double().numpy(), v.double().numpy(), causal=causal,
+                                   scale=d ** -0.5)
+    assert_close(o, lse, o_ref, lse_ref, f"B{B}H{H}N{N}d{d} causal={causal} x{mult}")
+
+
+def test_non_default_scale_and_seed():
+    q, k, v = make_qkv(1, 3, 300, 128, seed=7)
+    o, lse = run_gpu(q, k, v, True, scale=0.05)
+    o_ref, lse_ref = attention_ref(q.double().numpy(), k.double().numpy(), v.double().numpy(), causal=True,
+                                   scale=0.05)
+    assert_close(o, lse, o_ref, lse_ref)
+
+
+def _sample_rows(N, rng, extra=12):
+    rows = {0, N - 1}
+    for t in (127, 128, 129, 255, 256, N // 2 - 1, N // 2, N - 128, N - 129):
+        if 0 <= t < N:
+            rows.add(t)
+    rows.update(rng.integers(0, N, size=extra).tolist())
+    return sorted(rows)
+
+
+FULL = ["B8_H16_N2048_d128_causal", "B1_H16_N16384_d128_causal",
+        "sweep_N512_d64_full", "sweep_N2048_d64_full", "sweep_N16384_d64_full",
+        "grid_N4096_d128_full", "grid_N8192_d64_causal", "grid_N1024_d128_causal"]
+
+
+@pytest.mark.parametrize("name", FULL)
+@pytest.mark.parametrize("mult", [1.0, 4.0], ids=["x1", "x4"])
+def test_full_size_sampled_rows(name, mult):
+    w = WORKLOADS[name]
+    q, k, v = make_qkv(w.B, w.H, w.N, w.d, seed=0, qk_mult=mult)
+    o_d, lse_d = fwd(q.cuda(), k.cuda(), v.cuda(), causal=w.causal)
+    sync_status()
+    assert torch.isfinite(lse_d).all().item()
+    assert torch.isfinite(o_d.float()).all().item()
+    o_all, lse_all = o_d.cpu(), lse_d.cpu()
+    rng = np.random.default_rng(1)
+    heads = {(0, 0), (w.B - 1, w.H - 1), (int(rng.integers(w.B)), int(rng.integers(w.H)))}
+    for b, h in sorted(heads):
+        rows = _sample_rows(w.N, rng)
+        o_ref, lse_ref = attention_ref_rows(q[b:b + 1, h:h + 1].double().numpy(), k[b:b + 1, h:h + 1].double().numpy(),
+                                            v[b:b + 1, h:h + 1].double().numpy(), 0, 0, rows, causal=w.causal,
+                                            scale=w.d ** -0.5)
+        assert_close(o_all[b, h, rows].double().numpy(), lse_all[b, h, rows].double().numpy(), o_ref, lse_ref,
+                     f"{name} x{mult} head ({b},{h})")
+
+
+def test_constant_v_gives_constant_output():
+    q, k, _ = make_qkv(2, 2, 515, 128, seed=3, qk_mult=2.0)
+    v = torch.full_like(q, 0.75)
+    for causal in (False, True):
+        o, _ = run_gpu(q, k, v, causal)
+        assert np.abs(o - 0.75).max() <= O_TOL
+
+
+def test_causal_row0_is_v0_exactly():
+    q, k, v = make_qkv(2, 3, 700, 64, seed=4)
+    o, lse = run_gpu(q, k, v, True)
+    assert np.array_equal(o[:, :, 0], v[:, :, 0].double().numpy())
+
+
+def test_causal_last_row_equals_full_last_row():
+    q, k, v = make_qkv(1, 2, 384, 128, seed=5)
+    oc, lc = run_gpu(q, k, v, True)
+    of, lf = run_gpu(q, k, v, False)
+    assert np.abs(oc[:, :, -1] - of[:, :, -1]).max() <= 1e-2
+    assert np.abs(lc[:, :, -1] - lf[:, :, -1]).max() <= 1e-3
+
+
+def test_repeatable_bitwise():
+    q, k, v = (t.cuda() for t in make_qkv(2, 4, 1024, 128, seed=6))
+    o1, l1 = fwd(q, k, v, causal=True)
+    o2, l2 = fwd(q, k, v, causal=True)
+    sync_status()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_side_stream_and_host_entry_agree():
+    q, k, v = make_qkv(2, 2, 640, 64, seed=8)
+    s = torch.cuda.Stream()
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        o1, l1 = fwd(qd, kd, vd, causal=False)
+    sync_status(s)
+    o2, l2 = fwd_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), causal=False)
+    assert torch.equal(o1.cpu(), o2) and torch.equal(l1.cpu(), l2)
