@@ -82,6 +82,26 @@ def recorded_traffic(workload: str, src_hash: str):
     return None
 
 
+def max_over_ranks(x: float, device) -> float:
+    """Maximum of a per-rank scalar over all ranks (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(flops_per_rank: float, world: int, max_ms_per_step: float) -> float:
+    """Whole-job throughput: every rank's FLOPs over the slowest rank's step time."""
+    return flops_per_rank * world / (max_ms_per_step * 1e-3) / 1e12
+
+
+def shard_seed(rank: int) -> int:
+    """Each rank draws its own shard of sequences."""
+    return int(rank)
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -235,7 +255,7 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     # Each rank draws its own shard of sequences (seed = rank) and keeps it resident.
-    q_h, k_h, v_h = make_qkv(w.B, w.H, w.N, w.d, seed=rank, qk_mult=w.qk_mult)
+    q_h, k_h, v_h = make_qkv(w.B, w.H, w.N, w.d, seed=shard_seed(rank), qk_mult=w.qk_mult)
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
@@ -288,13 +308,10 @@ def main():
     barrier()
     fa2.sync_status(stream)
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(total_ms, dev)
     ms_per_step = max_ms / args.steps
     total_flops = w.flops * world
-    value = total_flops / (ms_per_step * 1e-3) / 1e12
+    value = aggregate_tflops(w.flops, world, ms_per_step)
 
     # End to end through the host-buffer entry point: pinned host inputs in,
     # host outputs back, copies inside the timed region.
@@ -314,11 +331,8 @@ def main():
             fa2.fwd_host(qp, kp, vp, causal=w.causal, out=op, lse=lp, workspace=ws, stream=stream)
         ev1.record(stream)
         torch.cuda.synchronize(dev)
-        te = torch.tensor([ev0.elapsed_time(ev1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te.item()) / e2e_steps
-        e2e = {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), dev) / e2e_steps
+        e2e = {"value": aggregate_tflops(w.flops, world, e2e_ms), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes, "steps": e2e_steps}
         del qp, kp, vp, op, lp, ws
 
