@@ -10,7 +10,8 @@
 //          1/l normalisation is deferred to the epilogue, exponentials use exp2
 //          with the softmax scale folded into one FMA, and only the diagonal
 //          (causal) or ragged tail tile is masked element by element;
-//      (2) parallel over the sequence: one CTA per (query tile, head, batch);
+//      (2) parallel over the sequence: one CTA per (256-row query block, head,
+//          batch);
 //      (3) work split without shared-memory reductions: each softmax thread
 //          owns one query row (one TMEM lane) from scores to output.
 //  * iplexlaw blog, section "Tiling preserves the attention calculation":
@@ -18,15 +19,20 @@
 //    rescales partial outputs so the result is the globally normalised one.
 //
 // B200 design (not in the pages, which describe A100 kernels):
-//  * warp 4 = TMA producer (Q once; K and V through separate rings);
-//  * warp 5 = MMA issuer: S_j = Q K_j^T (SS form) into one of two TMEM score
-//    buffers, O += P_j V_j (TS form: P read from TMEM), commits to mbarriers;
-//  * warps 0-3 = softmax / correction / epilogue, thread t <-> query row t
-//    <-> TMEM lane t;
+//  * a CTA owns two 128-row query tiles (t = 0, 1) that share every K/V tile;
+//    the tensor core works on one tile while the softmax warpgroup of the
+//    other tile computes exponentials (ping-pong);
+//  * warp 8 = TMA producer (Q0, Q1 once; K and V through separate rings);
+//  * warp 9 = MMA issuer.  Per K/V tile j it issues
+//        PV_0(j-1), S_0(j), PV_1(j-1), S_1(j)
+//    with S_t = Q_t K_j^T (both operands in shared memory) into tile t's TMEM
+//    score columns and O_t += P_t V (P read from TMEM, V from shared memory);
+//  * warpgroup t (warps 4t..4t+3) = softmax of tile t: thread r <-> query row
+//    r <-> TMEM lane r.  P (bf16) is written over the first 64 score columns;
 //  * the O rescale is skipped unless a row's running max grows by more than
 //    RESCALE_THRESHOLD (log2 units).  The stale max is used consistently for
 //    P, the running sum and the final LSE, so the result is unchanged (the
-//    exponentials stay below 2^RESCALE_THRESHOLD).
+//    exponentials stay below 2^RESCALE_THRESHOLD);
 //  * every wait is bounded; on time-out the kernel records a status word,
 //    drains its own in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -47,17 +53,25 @@ namespace fa2 {
 
 using namespace ptx;
 
-constexpr int BM = 128;  // query rows per CTA (one tcgen05 M=128 tile)
-constexpr int BN = 128;  // keys per K/V tile
-constexpr int NUM_THREADS = 192;
-constexpr int PRODUCER_WARP = 4;
-constexpr int MMA_WARP = 5;
+constexpr int BM = 128;         // query rows per tile (one tcgen05 M=128 MMA)
+constexpr int Q_TILES = 2;      // query tiles per CTA
+constexpr int BLOCK_M = BM * Q_TILES;
+constexpr int BN = 128;         // keys per K/V tile
+constexpr int NUM_THREADS = 384;
+constexpr int PRODUCER_WARP = 8;
+constexpr int MMA_WARP = 9;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_S0 = 0;    // score buffer 0: 128 fp32 columns
-constexpr uint32_t TM_S1 = 128;  // score buffer 1
-constexpr uint32_t TM_P = 256;   // probabilities: 128 bf16 per row = 64 columns
-constexpr uint32_t TM_O = 384;   // output accumulator: d fp32 columns
+// TMEM columns of tile t: scores at 128*t (P aliases the first 64 of them),
+// output accumulator at 256 + 128*t.
+__host__ __device__ constexpr uint32_t tm_s(int t) { return 128u * static_cast<uint32_t>(t); }
+__host__ __device__ constexpr uint32_t tm_o(int t) { return 256u + 128u * static_cast<uint32_t>(t); }
 constexpr float RESCALE_THRESHOLD = 8.0f;
+// Register split: launched at 168 per thread (384 threads), the softmax
+// warpgroups grow to 208 and the control warpgroup shrinks to 80:
+// 256*208 + 128*80 = 63488 <= 384*168 = 64512.
+constexpr uint32_t REGS_SOFTMAX = 208;
+constexpr uint32_t REGS_CONTROL = 80;
+static_assert(256 * REGS_SOFTMAX + 128 * REGS_CONTROL <= 384 * 168, "register split exceeds the launch budget");
 
 // Device status word: bit 0 = a bounded wait gave up; bits 8..11 = role.
 __device__ unsigned int g_fa2_status = 0;
@@ -68,13 +82,13 @@ constexpr unsigned int ROLE_PRODUCER = 1u << 8, ROLE_MMA = 2u << 8, ROLE_SOFTMAX
 template <int HD>
 struct Cfg {
   static_assert(HD == 64 || HD == 128, "head dimension");
-  static constexpr int KCH = HD / 64;                  // 64-element (128-byte) column chunks
-  static constexpr int CHUNK_BYTES = 128 * 128;        // 128 rows x 128 bytes
+  static constexpr int KCH = HD / 64;                   // 64-element (128-byte) column chunks
+  static constexpr int CHUNK_BYTES = 128 * 128;         // 128 rows x 128 bytes
   static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;  // one 128-row Q/K/V tile
-  static constexpr int KS = (HD == 128) ? 2 : 3;       // K ring stages
-  static constexpr int VS = (HD == 128) ? 2 : 3;       // V ring stages
+  static constexpr int KS = (HD == 128) ? 2 : 3;        // K ring stages
+  static constexpr int VS = (HD == 128) ? 2 : 3;        // V ring stages
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + TILE_BYTES;
+  static constexpr int OFF_K = OFF_Q + Q_TILES * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + VS * TILE_BYTES;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
@@ -86,24 +100,25 @@ struct Params {
   float* lse;
   int N;
   int H;
-  int n_q_tiles;
-  int n_kv_tiles;
+  int n_q_blocks;  // 256-row query blocks
+  int n_kv_tiles;  // 128-key tiles
   float scale_log2;  // scale * log2(e)
   unsigned long long timeout_ns;
-  int inject_timeout;  // test hook: withhold the Q load
+  int inject_timeout;  // test hook: withhold the Q loads
 };
 
 struct Barriers {
-  uint64_t q_full;
+  uint64_t q_full[2];
   uint64_t k_full[3], k_empty[3];
   uint64_t v_full[3], v_empty[3];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full;
-  uint64_t pv_done;
+  uint64_t s_full[2];   // S_t(j) complete (and every MMA issued before it)
+  uint64_t p_full[2];   // softmax t wrote P_t(j) (and rescaled O_t if needed)
+  uint64_t o_ready[2];  // last PV_t complete
   uint64_t mma_final;
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(Barriers) <= 256, "barrier block");
 
 // Bounded wait.  Returns false (and records the time-out once) if the phase
 // did not complete within timeout_ns, or if another role already gave up.
@@ -124,6 +139,13 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
   }
 }
 
+// Warp-uniform bounded wait for the softmax warps (all 32 lanes agree).
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long timeout_ns) {
+  const bool ok = wait_bounded(bar, parity, abort_flag, timeout_ns, ROLE_SOFTMAX);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Bounded wait used while draining: ignores the abort flag.
 __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, unsigned long long timeout_ns) {
   const uint64_t t0 = globaltimer_ns();
@@ -134,6 +156,150 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, unsign
     }
   }
   return true;
+}
+
+// Number of K/V tiles query tile t of block qb attends to.
+template <bool CAUSAL>
+__device__ __forceinline__ int kv_tiles_for(int qb, int t, int n_kv_tiles) {
+  if (!CAUSAL) return n_kv_tiles;
+  return min(qb * Q_TILES + t + 1, n_kv_tiles);  // the diagonal tile is the last one
+}
+
+// ------------------------------------------------------------------ softmax
+// One thread = one query row of tile t.  Returns false if a wait gave up.
+template <int HD, bool CAUSAL>
+__device__ __forceinline__ void softmax_role(const Params& p, Barriers* bars, volatile int* abort_flag,
+                                             uint32_t tmem, int t, int warp_in_wg, int lane, int row_g, int bh,
+                                             int n_t) {
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp_in_wg * 32) << 16);
+  const uint32_t s_addr = lane_base + tm_s(t);
+  const uint32_t o_addr = lane_base + tm_o(t);
+  const uint32_t b_s = smem_u32(&bars->s_full[t]);
+  const uint32_t b_p = smem_u32(&bars->p_full[t]);
+  const float c_log2 = p.scale_log2;
+  const uint64_t cc = f2_pack(c_log2, c_log2);
+  const int q_first = row_g - (warp_in_wg * 32 + lane);  // first row of this tile
+  float m = -INFINITY;  // running max of scale*log2(e)*s (possibly stale, see header)
+  float l = 0.f;        // running sum of exp2(...) relative to m
+  bool ok = true;
+  for (int j = 0; j < n_t; ++j) {
+    ok = wait_warp(b_s, j & 1, abort_flag, p.timeout_ns);
+    if (!ok) break;
+    tc_fence_after();
+    uint32_t s[128];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
+
+    const int kv0 = j * BN;
+    const bool diag = CAUSAL && (kv0 + BN - 1 > q_first);  // tile reaches past this tile's first row
+    const bool tail = !CAUSAL && (kv0 + BN > p.N);          // ragged last key tile
+    if (diag || tail) {
+      const int lim = diag ? (row_g - kv0) : (p.N - 1 - kv0);  // last allowed column
+#pragma unroll
+      for (int e = 0; e < 128; ++e)
+        if (e > lim) s[e] = __float_as_uint(-INFINITY);
+    }
+    // Row max: eight independent 3-input chains, then combine.
+    float mx8[8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a) mx8[a] = __uint_as_float(s[a]);
+#pragma unroll
+    for (int e = 8; e < 128; e += 16)
+#pragma unroll
+      for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], __uint_as_float(s[e + a]), __uint_as_float(s[e + 8 + a]));
+    const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+    const float m_cand = mx * c_log2;
+    float m_new = m;
+    if (m_cand > m + RESCALE_THRESHOLD) m_new = m_cand;  // also taken on the first tile (m = -inf)
+    const bool rescale = (j > 0) && (m_new != m);
+    const float alpha = rescale ? ex2(m - m_new) : 1.f;
+    const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+    const uint64_t mm = f2_pack(-m_use, -m_use);
+
+    // p = exp2(s*c - m): one packed FMA per pair, ex2 per element; P packed to
+    // bf16 and written over the score columns 32 at a time.
+    uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t pk[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int i = h * 64 + 2 * e;
+        const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), cc, mm);
+        float x0, x1;
+        f2_unpack(x, x0, x1);
+        const float p0 = ex2(x0), p1 = ex2(x1);
+        acc[e & 3] = f2_add(acc[e & 3], f2_pack(p0, p1));
+        pk[e] = pack_bf16x2(p0, p1);
+      }
+      tmem_st32(s_addr + h * 32, pk);
+    }
+    float r0, r1, r2, r3, r4, r5, r6, r7;
+    f2_unpack(f2_add(acc[0], acc[1]), r0, r1);
+    f2_unpack(f2_add(acc[2], acc[3]), r2, r3);
+    (void)r4; (void)r5; (void)r6; (void)r7;
+    const float rowsum = (r0 + r1) + (r2 + r3);
+
+    // S_t(j) complete implies PV_t(j-1) complete (the commit tracks every
+    // earlier MMA), so O_t is stable here.
+    if (__any_sync(0xffffffffu, rescale)) {
+      const uint64_t aa = f2_pack(alpha, alpha);
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(o_addr + c * 32, o);
+        tmem_wait_ld();
+        reg_fence32(o);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float a0, a1;
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), aa), a0, a1);
+          o[e] = __float_as_uint(a0);
+          o[e + 1] = __float_as_uint(a1);
+        }
+        tmem_st32(o_addr + c * 32, o);
+      }
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(b_p);
+    l = l * alpha + rowsum;
+    m = m_new;
+  }
+  if (ok) ok = wait_warp(smem_u32(&bars->o_ready[t]), 0, abort_flag, p.timeout_ns);
+  if (!ok) return;
+  tc_fence_after();
+  const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+  const bool store = row_g < p.N;
+  __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (store ? row_g : 0)) * HD;
+  const uint64_t il = f2_pack(inv_l, inv_l);
+#pragma unroll
+  for (int c = 0; c < HD / 32; ++c) {
+    uint32_t o[32];
+    tmem_ld32(o_addr + c * 32, o);
+    tmem_wait_ld();
+    reg_fence32(o);
+    uint32_t w[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      float a0, a1;
+      f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), il), a0, a1);
+      w[e] = pack_bf16x2(a0, a1);
+    }
+    if (store) {
+      uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+    }
+  }
+  if (store) {
+    const float lse = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    p.lse[static_cast<size_t>(bh) * p.N + row_g] = lse;
+  }
 }
 
 template <int HD, bool CAUSAL>
@@ -156,18 +322,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int qt = CAUSAL ? (p.n_q_tiles - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+  const int qb = CAUSAL ? (p.n_q_blocks - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
   const int bh = static_cast<int>(blockIdx.z) * p.H + static_cast<int>(blockIdx.y);
-  const int q0 = qt * BM;
-  const int nkv = CAUSAL ? min(qt + 1, p.n_kv_tiles) : p.n_kv_tiles;
-
-  const uint32_t b_q_full = smem_u32(&bars->q_full);
-  const uint32_t b_pfull = smem_u32(&bars->p_full);
-  const uint32_t b_pvdone = smem_u32(&bars->pv_done);
-  const uint32_t b_final = smem_u32(&bars->mma_final);
+  const int q0 = qb * BLOCK_M;
+  const int n0 = kv_tiles_for<CAUSAL>(qb, 0, p.n_kv_tiles);
+  const int n1 = kv_tiles_for<CAUSAL>(qb, 1, p.n_kv_tiles);  // n0 <= n1
 
   if (threadIdx.x == 0) {
-    mbar_init(b_q_full, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(smem_u32(&bars->q_full[t]), 1);
+      mbar_init(smem_u32(&bars->s_full[t]), 1);
+      mbar_init(smem_u32(&bars->p_full[t]), 4);
+      mbar_init(smem_u32(&bars->o_ready[t]), 1);
+    }
     for (int s = 0; s < C::KS; ++s) {
       mbar_init(smem_u32(&bars->k_full[s]), 1);
       mbar_init(smem_u32(&bars->k_empty[s]), 1);
@@ -176,13 +343,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&bars->v_full[s]), 1);
       mbar_init(smem_u32(&bars->v_empty[s]), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(smem_u32(&bars->s_full[s]), 1);
-      mbar_init(smem_u32(&bars->s_free[s]), 4);
-    }
-    mbar_init(b_pfull, 4);
-    mbar_init(b_pvdone, 1);
-    mbar_init(b_final, 1);
+    mbar_init(smem_u32(&bars->mma_final), 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -200,16 +361,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == PRODUCER_WARP) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+  if (warp >= 8) {
+    regs_dec<REGS_CONTROL>();
+    if (warp == PRODUCER_WARP && lane == 0) {
+      // ---------------------------------------------------------- TMA producer
       const bool load_q = !p.inject_timeout;
       if (load_q) {
-        mbar_arrive_expect_tx(b_q_full, C::TILE_BYTES);
-        for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * C::CHUNK_BYTES, &tm_q, b_q_full, c * 64, q0, bh);
+        for (int t = 0; t < 2; ++t) {
+          // A tile that starts at or past N has no row to store; it is loaded
+          // from tile 0's rows so that no copy lies wholly outside the tensor.
+          const int qy = (q0 + t * BM < p.N) ? q0 + t * BM : q0;
+          const uint32_t qbar = smem_u32(&bars->q_full[t]);
+          mbar_arrive_expect_tx(qbar, C::TILE_BYTES);
+          for (int c = 0; c < C::KCH; ++c)
+            tma_load_3d(sQ + t * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, qbar, c * 64, qy, bh);
+        }
       }
       int k_issued = 0, v_issued = 0;
-      for (int j = 0; j < nkv; ++j) {
+      for (int j = 0; j < n1; ++j) {
         const int ks = j % C::KS;
         if (j >= C::KS &&
             !wait_bounded(smem_u32(&bars->k_empty[ks]), ((j / C::KS) - 1) & 1, abort_flag, p.timeout_ns,
@@ -232,179 +401,105 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++v_issued;
       }
       // Drain: every load this thread issued must land before the CTA exits.
-      if (load_q) wait_drain(b_q_full, 0, p.timeout_ns);
+      if (load_q) {
+        wait_drain(smem_u32(&bars->q_full[0]), 0, p.timeout_ns);
+        wait_drain(smem_u32(&bars->q_full[1]), 0, p.timeout_ns);
+      }
       for (int t = (k_issued > C::KS ? k_issued - C::KS : 0); t < k_issued; ++t)
         wait_drain(smem_u32(&bars->k_full[t % C::KS]), (t / C::KS) & 1, p.timeout_ns);
       for (int t = (v_issued > C::VS ? v_issued - C::VS : 0); t < v_issued; ++t)
         wait_drain(smem_u32(&bars->v_full[t % C::VS]), (t / C::VS) & 1, p.timeout_ns);
-    }
-  } else if (warp == MMA_WARP) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == MMA_WARP && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
-      bool ok = wait_bounded(b_q_full, 0, abort_flag, p.timeout_ns, ROLE_MMA);
-      for (int j = 0; ok && j <= nkv; ++j) {
-        if (j < nkv) {
-          const int ks = j % C::KS;
-          const int sb = j & 1;
-          if (!wait_bounded(smem_u32(&bars->k_full[ks]), (j / C::KS) & 1, abort_flag, p.timeout_ns, ROLE_MMA))
-            break;
-          if (j >= 2 &&
-              !wait_bounded(smem_u32(&bars->s_free[sb]), ((j - 2) >> 1) & 1, abort_flag, p.timeout_ns, ROLE_MMA))
-            break;
-          tc_fence_after();
-          const uint32_t d_s = tmem + (sb ? TM_S1 : TM_S0);
-          const uint32_t kbase = sK + ks * C::TILE_BYTES;
+      auto issue_s = [&](int t, int ks) {
+        const uint32_t qbase = sQ + t * C::TILE_BYTES;
+        const uint32_t kbase = sK + ks * C::TILE_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-            mma_ss(d_s, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024), IDESC_S,
-                   kk > 0 ? 1u : 0u);
-          }
-          mma_commit(smem_u32(&bars->s_full[sb]));
-          mma_commit(smem_u32(&bars->k_empty[ks]));
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+          mma_ss(tmem + tm_s(t), smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
+                 IDESC_S, kk > 0 ? 1u : 0u);
         }
-        if (j >= 1) {
-          const int i = j - 1;
-          const int vs = i % C::VS;
-          if (!wait_bounded(b_pfull, i & 1, abort_flag, p.timeout_ns, ROLE_MMA)) break;
-          if (!wait_bounded(smem_u32(&bars->v_full[vs]), (i / C::VS) & 1, abort_flag, p.timeout_ns, ROLE_MMA))
-            break;
-          tc_fence_after();
-          const uint32_t vbase = sV + vs * C::TILE_BYTES;
+      };
+      auto issue_pv = [&](int t, int vs, bool acc) {
+        const uint32_t vbase = sV + vs * C::TILE_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            mma_ts(tmem + TM_O, tmem + TM_P + kk * 8, smem_desc_sw128(vbase + kk * 2048, C::CHUNK_BYTES, 1024),
-                   IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(smem_u32(&bars->v_empty[vs]));
-          mma_commit(b_pvdone);
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(tmem + tm_o(t), tmem + tm_s(t) + kk * 8,
+                 smem_desc_sw128(vbase + kk * 2048, C::CHUNK_BYTES, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+      };
+      const unsigned long long to = p.timeout_ns;
+      bool ok = true;
+      // K/V tile 0: S_0(0), S_1(0).
+      ok = wait_bounded(smem_u32(&bars->q_full[0]), 0, abort_flag, to, ROLE_MMA) &&
+           wait_bounded(smem_u32(&bars->k_full[0]), 0, abort_flag, to, ROLE_MMA);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        mma_commit(smem_u32(&bars->s_full[0]));
+        ok = wait_bounded(smem_u32(&bars->q_full[1]), 0, abort_flag, to, ROLE_MMA);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_s(1, 0);
+        mma_commit(smem_u32(&bars->s_full[1]));
+        mma_commit(smem_u32(&bars->k_empty[0]));
+      }
+      // Steady state and tail: iteration j issues the PVs of tile j-1 and
+      // the scores of tile j.
+      for (int j = 1; ok && j <= n1; ++j) {
+        const int i = j - 1;  // K/V tile whose PV is issued now
+        const int vs = i % C::VS;
+        const int ks = j % C::KS;
+        bool v_ready = false;
+        // tile 0
+        if (i < n0) {
+          ok = wait_bounded(smem_u32(&bars->p_full[0]), i & 1, abort_flag, to, ROLE_MMA) &&
+               wait_bounded(smem_u32(&bars->v_full[vs]), (i / C::VS) & 1, abort_flag, to, ROLE_MMA);
+          if (!ok) break;
+          v_ready = true;
+          tc_fence_after();
+          issue_pv(0, vs, i > 0);
+          if (i == n0 - 1) mma_commit(smem_u32(&bars->o_ready[0]));
+        }
+        if (j < n0) {
+          ok = wait_bounded(smem_u32(&bars->k_full[ks]), (j / C::KS) & 1, abort_flag, to, ROLE_MMA);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(0, ks);
+          mma_commit(smem_u32(&bars->s_full[0]));
+        }
+        // tile 1
+        ok = wait_bounded(smem_u32(&bars->p_full[1]), i & 1, abort_flag, to, ROLE_MMA) &&
+             (v_ready || wait_bounded(smem_u32(&bars->v_full[vs]), (i / C::VS) & 1, abort_flag, to, ROLE_MMA));
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, vs, i > 0);
+        mma_commit(smem_u32(&bars->v_empty[vs]));
+        if (i == n1 - 1) mma_commit(smem_u32(&bars->o_ready[1]));
+        if (j < n1) {
+          ok = wait_bounded(smem_u32(&bars->k_full[ks]), (j / C::KS) & 1, abort_flag, to, ROLE_MMA);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(1, ks);
+          mma_commit(smem_u32(&bars->s_full[1]));
+          mma_commit(smem_u32(&bars->k_empty[ks]));
         }
       }
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
-      mma_commit(b_final);
-      wait_drain(b_final, 0, p.timeout_ns);
+      mma_commit(smem_u32(&bars->mma_final));
+      wait_drain(smem_u32(&bars->mma_final), 0, p.timeout_ns);
     }
   } else {
-    // ------------------------------------------------------------ softmax warps 0..3
-    const int r = threadIdx.x;  // query row within the tile == TMEM lane
-    const int row_g = q0 + r;
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const float c_log2 = p.scale_log2;
-    float m = -INFINITY;  // running max of scale*log2(e)*s (possibly stale, see header)
-    float l = 0.f;        // running sum of exp2(...) relative to m
-    bool ok = true;
-    for (int i = 0; i < nkv; ++i) {
-      const int sb = i & 1;
-      ok = wait_bounded(smem_u32(&bars->s_full[sb]), (i >> 1) & 1, abort_flag, p.timeout_ns, ROLE_SOFTMAX);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t s[4][32];
-      const uint32_t s_addr = lane_addr + (sb ? TM_S1 : TM_S0);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, s[c]);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence32(s[c]);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[sb]));
-
-      const int kv0 = i * BN;
-      const bool diag = CAUSAL && (kv0 + BN > q0);       // tile reaches past this CTA's first row
-      const bool tail = !CAUSAL && (kv0 + BN > p.N);     // ragged last key tile
-      if (diag || tail) {
-        const int lim = diag ? (row_g - kv0) : (p.N - 1 - kv0);  // last allowed column
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c * 32 + e > lim) s[c][e] = __float_as_uint(-INFINITY);
-      }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(s[c][e]));
-      const float m_cand = mx * c_log2;
-      float m_new = m;
-      if (m_cand > m + RESCALE_THRESHOLD) m_new = m_cand;  // also taken on the first tile (m = -inf)
-      const bool rescale = (i > 0) && (m_new != m);
-      const float alpha = rescale ? ex2(m - m_new) : 1.f;
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-
-      float rowsum = 0.f;
-      uint32_t pk[2][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float p0 = ex2(fmaf(__uint_as_float(s[c][e]), c_log2, -m_use));
-          const float p1 = ex2(fmaf(__uint_as_float(s[c][e + 1]), c_log2, -m_use));
-          rowsum += p0 + p1;
-          pk[c >> 1][(c & 1) * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
-        }
-      }
-      if (i > 0) {
-        // O and the P buffer are in use by PV_{i-1} until it completes.
-        ok = wait_bounded(b_pvdone, (i - 1) & 1, abort_flag, p.timeout_ns, ROLE_SOFTMAX);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-          for (int c = 0; c < HD / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(lane_addr + TM_O + c * 32, o);
-            tmem_wait_ld();
-            reg_fence32(o);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(lane_addr + TM_O + c * 32, o);
-          }
-        }
-      }
-      tmem_st32(lane_addr + TM_P, pk[0]);
-      tmem_st32(lane_addr + TM_P + 32, pk[1]);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(b_pfull);
-      l = l * alpha + rowsum;
-      m = m_new;
-    }
-    if (ok && nkv > 0) {
-      ok = wait_bounded(b_pvdone, (nkv - 1) & 1, abort_flag, p.timeout_ns, ROLE_SOFTMAX);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
-      tc_fence_after();
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const bool store = row_g < p.N;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (store ? row_g : 0)) * HD;
-#pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(lane_addr + TM_O + c * 32, o);
-        tmem_wait_ld();
-        reg_fence32(o);
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-        }
-      }
-      if (store) {
-        const float lse = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-        p.lse[static_cast<size_t>(bh) * p.N + row_g] = lse;
-      }
-    }
+    // ------------------------------------------------------------ softmax warpgroups
+    regs_inc<REGS_SOFTMAX>();
+    const int t = warp >> 2;            // query tile of this warpgroup
+    const int warp_in_wg = warp & 3;    // TMEM lane quadrant
+    const int r = warp_in_wg * 32 + lane;
+    const int row_g = q0 + t * BM + r;
+    softmax_role<HD, CAUSAL>(p, bars, abort_flag, tmem, t, warp_in_wg, lane, row_g, bh, t == 0 ? n0 : n1);
   }
 
   tc_fence_before();
@@ -519,7 +614,7 @@ static int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
     }
     if (dev < 32) attr_done_mask |= (1 << dev);
   }
-  dim3 grid(prm.n_q_tiles, H, B);
+  dim3 grid(prm.n_q_blocks, H, B);
   kern<<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -544,7 +639,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   prm.lse = lse;
   prm.N = N;
   prm.H = H;
-  prm.n_q_tiles = (N + BM - 1) / BM;
+  prm.n_q_blocks = (N + BLOCK_M - 1) / BLOCK_M;
   prm.n_kv_tiles = (N + BN - 1) / BN;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
   prm.timeout_ns = timeout_ns;
