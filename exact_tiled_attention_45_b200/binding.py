@@ -14,7 +14,8 @@ import os
 import torch
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG_DIR, "libfa2.so")
+#: The in-tree build; FA2_LIBRARY may name another build of the same sources.
+LIB_PATH = os.environ.get("FA2_LIBRARY") or os.path.join(_PKG_DIR, "libfa2.so")
 
 FA2_OK, FA2_ERR_INVALID_ARG, FA2_ERR_UNSUPPORTED, FA2_ERR_CUDA, FA2_ERR_TIMEOUT = range(5)
 

@@ -66,12 +66,36 @@ constexpr uint32_t TMEM_COLS = 512;
 __host__ __device__ constexpr uint32_t tm_s(int t) { return 128u * static_cast<uint32_t>(t); }
 __host__ __device__ constexpr uint32_t tm_o(int t) { return 256u + 128u * static_cast<uint32_t>(t); }
 constexpr float RESCALE_THRESHOLD = 8.0f;
+#ifndef FA2_EMU_PAIRS_D128
+#define FA2_EMU_PAIRS_D128 2
+#endif
+#ifndef FA2_EMU_PAIRS_D64
+#define FA2_EMU_PAIRS_D64 3
+#endif
 // Register split: launched at 168 per thread (384 threads), the softmax
-// warpgroups grow to 208 and the control warpgroup shrinks to 80:
-// 256*208 + 128*80 = 63488 <= 384*168 = 64512.
-constexpr uint32_t REGS_SOFTMAX = 208;
-constexpr uint32_t REGS_CONTROL = 80;
+// warpgroups grow to 216 and the control warpgroup shrinks to 64:
+// 256*216 + 128*64 = 63488 <= 384*168 = 64512.
+constexpr uint32_t REGS_SOFTMAX = 216;
+constexpr uint32_t REGS_CONTROL = 64;
 static_assert(256 * REGS_SOFTMAX + 128 * REGS_CONTROL <= 384 * 168, "register split exceeds the launch budget");
+
+// Optional per-role timeline (compile with -DFA2_TRACE): SM clock stamps of
+// the pipeline events of CTA (0,0,0), read back with fa2_trace_read().  The
+// product build compiles every stamp away.
+#ifdef FA2_TRACE
+constexpr int TRACE_J = 64;   // K/V tiles recorded
+constexpr int TRACE_EV = 24;  // event kinds
+__device__ long long g_fa2_trace[TRACE_EV * TRACE_J + 1];
+#define FA2_STAMP(ev, j)                                                                          \
+  do {                                                                                            \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (j) >= 0 && (j) < TRACE_J)        \
+      g_fa2_trace[(ev) * TRACE_J + (j)] = clock64();                                              \
+  } while (0)
+#else
+#define FA2_STAMP(ev, j) \
+  do {                   \
+  } while (0)
+#endif
 
 // Device status word: bit 0 = a bounded wait gave up; bits 8..11 = role.
 __device__ unsigned int g_fa2_status = 0;
@@ -87,6 +111,10 @@ struct Cfg {
   static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;  // one 128-row Q/K/V tile
   static constexpr int KS = (HD == 128) ? 2 : 3;        // K ring stages
   static constexpr int VS = (HD == 128) ? 2 : 3;        // V ring stages
+  // Of every 8 pairs of scores, this many are exponentiated on the FMA pipe
+  // (polynomial) and the rest on the special-function unit.  At d = 128 the
+  // special-function work of a tile equals its MMA time; at d = 64 it is twice.
+  static constexpr int EMU_PAIRS_PER_8 = (HD == 128) ? FA2_EMU_PAIRS_D128 : FA2_EMU_PAIRS_D64;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_TILES * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
@@ -114,7 +142,7 @@ struct Barriers {
   uint64_t s_full[2];   // S_t(j) complete (and every MMA issued before it)
   uint64_t p_full[2];   // softmax t wrote P_t(j) (and rescaled O_t if needed)
   uint64_t o_ready[2];  // last PV_t complete
-  uint64_t mma_final;
+  uint64_t mma_final[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -185,6 +213,7 @@ __device__ __forceinline__ void softmax_role(const Params& p, Barriers* bars, vo
   for (int j = 0; j < n_t; ++j) {
     ok = wait_warp(b_s, j & 1, abort_flag, p.timeout_ns);
     if (!ok) break;
+    if (lane == 0 && warp_in_wg < 2) FA2_STAMP(warp_in_wg == 0 ? 12 + 6 * t : 22 + t, j);
     tc_fence_after();
     uint32_t s[128];
 #pragma unroll
@@ -229,9 +258,15 @@ __device__ __forceinline__ void softmax_role(const Params& p, Barriers* bars, vo
       for (int e = 0; e < 32; ++e) {
         const int i = h * 64 + 2 * e;
         const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), cc, mm);
-        float x0, x1;
-        f2_unpack(x, x0, x1);
-        const float p0 = ex2(x0), p1 = ex2(x1);
+        float p0, p1;
+        if (((h * 32 + e) & 7) < Cfg<HD>::EMU_PAIRS_PER_8) {
+          f2_unpack(exp2_poly_pair(x), p0, p1);  // FMA pipe
+        } else {
+          float x0, x1;
+          f2_unpack(x, x0, x1);
+          p0 = ex2(x0);  // special-function unit
+          p1 = ex2(x1);
+        }
         acc[e & 3] = f2_add(acc[e & 3], f2_pack(p0, p1));
         pk[e] = pack_bf16x2(p0, p1);
       }
@@ -245,6 +280,7 @@ __device__ __forceinline__ void softmax_role(const Params& p, Barriers* bars, vo
 
     // S_t(j) complete implies PV_t(j-1) complete (the commit tracks every
     // earlier MMA), so O_t is stable here.
+    if (warp_in_wg == 0 && lane == 0) FA2_STAMP(13 + 6 * t, j);
     if (__any_sync(0xffffffffu, rescale)) {
       const uint64_t aa = f2_pack(alpha, alpha);
 #pragma unroll
@@ -267,6 +303,7 @@ __device__ __forceinline__ void softmax_role(const Params& p, Barriers* bars, vo
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(b_p);
+    if (lane == 0) FA2_STAMP(8 + 6 * t + warp_in_wg, j);
     l = l * alpha + rowsum;
     m = m_new;
   }
@@ -343,7 +380,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&bars->v_full[s]), 1);
       mbar_init(smem_u32(&bars->v_empty[s]), 1);
     }
-    mbar_init(smem_u32(&bars->mma_final), 1);
+    mbar_init(smem_u32(&bars->mma_final[0]), 1);
+    mbar_init(smem_u32(&bars->mma_final[1]), 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -360,6 +398,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+#ifdef FA2_TRACE
+  if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+    g_fa2_trace[TRACE_EV * TRACE_J] = clock64();
+#endif
 
   if (warp >= 8) {
     regs_dec<REGS_CONTROL>();
@@ -385,6 +427,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                           ROLE_PRODUCER))
           break;
         const uint32_t kb = smem_u32(&bars->k_full[ks]);
+        FA2_STAMP(20, j);
         mbar_arrive_expect_tx(kb, C::TILE_BYTES);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_3d(sK + ks * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_k, kb, c * 64, j * BN, bh);
@@ -395,6 +438,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                           ROLE_PRODUCER))
           break;
         const uint32_t vb = smem_u32(&bars->v_full[vs]);
+        FA2_STAMP(21, j);
         mbar_arrive_expect_tx(vb, C::TILE_BYTES);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_3d(sV + vs * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_v, vb, c * 64, j * BN, bh);
@@ -411,86 +455,85 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         wait_drain(smem_u32(&bars->v_full[t % C::VS]), (t / C::VS) & 1, p.timeout_ns);
     } else if (warp == MMA_WARP && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
+      // The tensor pipe keeps at most about one MMA queued, so the issuer does
+      // all of a step's waits first and then issues that step's MMAs back to
+      // back; every instruction between two MMAs is idle pipe time.
       constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
       auto issue_s = [&](int t, int ks) {
         const uint32_t qbase = sQ + t * C::TILE_BYTES;
         const uint32_t kbase = sK + ks * C::TILE_BYTES;
+        const uint32_t d_s = tmem + tm_s(t);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-          mma_ss(tmem + tm_s(t), smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
-                 IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss(d_s, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024), IDESC_S,
+                 kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int vs, bool acc) {
         const uint32_t vbase = sV + vs * C::TILE_BYTES;
+        const uint32_t d_o = tmem + tm_o(t), a_p = tmem + tm_s(t);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(tmem + tm_o(t), tmem + tm_s(t) + kk * 8,
-                 smem_desc_sw128(vbase + kk * 2048, C::CHUNK_BYTES, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(d_o, a_p + kk * 8, smem_desc_sw128(vbase + kk * 2048, C::CHUNK_BYTES, 1024), IDESC_PV,
+                 (acc || kk > 0) ? 1u : 0u);
       };
       const unsigned long long to = p.timeout_ns;
-      bool ok = true;
+      auto wait = [&](const uint64_t* bar, uint32_t parity) {
+        return wait_bounded(smem_u32(bar), parity, abort_flag, to, ROLE_MMA);
+      };
       // K/V tile 0: S_0(0), S_1(0).
-      ok = wait_bounded(smem_u32(&bars->q_full[0]), 0, abort_flag, to, ROLE_MMA) &&
-           wait_bounded(smem_u32(&bars->k_full[0]), 0, abort_flag, to, ROLE_MMA);
+      bool ok = wait(&bars->q_full[0], 0) && wait(&bars->k_full[0], 0);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
         mma_commit(smem_u32(&bars->s_full[0]));
-        ok = wait_bounded(smem_u32(&bars->q_full[1]), 0, abort_flag, to, ROLE_MMA);
+        FA2_STAMP(3, 0);
+        ok = wait(&bars->q_full[1], 0);
       }
       if (ok) {
-        tc_fence_after();
         issue_s(1, 0);
         mma_commit(smem_u32(&bars->s_full[1]));
         mma_commit(smem_u32(&bars->k_empty[0]));
+        FA2_STAMP(7, 0);
       }
-      // Steady state and tail: iteration j issues the PVs of tile j-1 and
-      // the scores of tile j.
+      // Step j: PV_0(j-1), S_0(j), PV_1(j-1), S_1(j).  Tile 0 may stop one
+      // K/V tile earlier (causal diagonal).
       for (int j = 1; ok && j <= n1; ++j) {
-        const int i = j - 1;  // K/V tile whose PV is issued now
+        const int i = j - 1;
         const int vs = i % C::VS;
         const int ks = j % C::KS;
-        bool v_ready = false;
-        // tile 0
-        if (i < n0) {
-          ok = wait_bounded(smem_u32(&bars->p_full[0]), i & 1, abort_flag, to, ROLE_MMA) &&
-               wait_bounded(smem_u32(&bars->v_full[vs]), (i / C::VS) & 1, abort_flag, to, ROLE_MMA);
-          if (!ok) break;
-          v_ready = true;
+        const bool do0 = i < n0, more0 = j < n0, more1 = j < n1;
+        FA2_STAMP(0, i);
+        ok = (!do0 || wait(&bars->p_full[0], i & 1)) && wait(&bars->v_full[vs], (i / C::VS) & 1) &&
+             (!more1 || wait(&bars->k_full[ks], (j / C::KS) & 1));
+        if (!ok) break;
+        FA2_STAMP(1, i);
+        if (do0) {
           tc_fence_after();
           issue_pv(0, vs, i > 0);
-          if (i == n0 - 1) mma_commit(smem_u32(&bars->o_ready[0]));
+          FA2_STAMP(2, i);
+          if (more0) issue_s(0, ks);
+          mma_commit(smem_u32(more0 ? &bars->s_full[0] : &bars->o_ready[0]));
+          FA2_STAMP(3, j);
         }
-        if (j < n0) {
-          ok = wait_bounded(smem_u32(&bars->k_full[ks]), (j / C::KS) & 1, abort_flag, to, ROLE_MMA);
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(0, ks);
-          mma_commit(smem_u32(&bars->s_full[0]));
-        }
-        // tile 1
-        ok = wait_bounded(smem_u32(&bars->p_full[1]), i & 1, abort_flag, to, ROLE_MMA) &&
-             (v_ready || wait_bounded(smem_u32(&bars->v_full[vs]), (i / C::VS) & 1, abort_flag, to, ROLE_MMA));
+        FA2_STAMP(4, i);
+        ok = wait(&bars->p_full[1], i & 1);
         if (!ok) break;
+        FA2_STAMP(5, i);
         tc_fence_after();
         issue_pv(1, vs, i > 0);
+        FA2_STAMP(6, i);
+        if (more1) issue_s(1, ks);
+        mma_commit(smem_u32(more1 ? &bars->s_full[1] : &bars->o_ready[1]));
         mma_commit(smem_u32(&bars->v_empty[vs]));
-        if (i == n1 - 1) mma_commit(smem_u32(&bars->o_ready[1]));
-        if (j < n1) {
-          ok = wait_bounded(smem_u32(&bars->k_full[ks]), (j / C::KS) & 1, abort_flag, to, ROLE_MMA);
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(1, ks);
-          mma_commit(smem_u32(&bars->s_full[1]));
-          mma_commit(smem_u32(&bars->k_empty[ks]));
-        }
+        if (more1) mma_commit(smem_u32(&bars->k_empty[ks]));
+        FA2_STAMP(7, j);
       }
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
-      mma_commit(smem_u32(&bars->mma_final));
-      wait_drain(smem_u32(&bars->mma_final), 0, p.timeout_ns);
+      mma_commit(smem_u32(&bars->mma_final[0]));
+      wait_drain(smem_u32(&bars->mma_final[0]), 0, p.timeout_ns);
     }
   } else {
     // ------------------------------------------------------------ softmax warpgroups
@@ -757,5 +800,16 @@ const char* fa2_strerror(int status) {
 const char* fa2_last_error_detail(void) { return fa2::g_detail; }
 
 int fa2_version(void) { return 100; }
+
+#ifdef FA2_TRACE
+// Trace builds only: copy the timeline ((24 events x 64 tiles) + start) to host.
+int fa2_trace_read(long long* host, int n) {
+  if (!host || n < fa2::TRACE_EV * fa2::TRACE_J + 1) return FA2_ERR_INVALID_ARG;
+  return cudaMemcpyFromSymbol(host, fa2::g_fa2_trace, sizeof(long long) * (fa2::TRACE_EV * fa2::TRACE_J + 1)) ==
+                 cudaSuccess
+             ? FA2_OK
+             : FA2_ERR_CUDA;
+}
+#endif
 
 }  // extern "C"

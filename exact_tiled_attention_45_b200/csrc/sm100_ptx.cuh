@@ -260,3 +260,42 @@ __device__ __forceinline__ void regs_dec() {
 }
 }  // namespace ptx
 }  // namespace fa2
+
+namespace fa2 {
+namespace ptx {
+// ---------------------------------------------------------------- 2^x on the FMA pipe
+// For a pair (x0, x1), x <= 2^22: 2^x = 2^j * 2^f with j = round(x) and
+// f = x - j in [-1/2, 1/2].  j comes from adding and subtracting 1.5 * 2^23
+// (round to nearest in fp32); 2^f is a degree-3 polynomial whose coefficients
+// were fitted for minimax relative error (fit_exp2_poly.py in this directory;
+// max relative error 1.0e-4 in fp32); 2^j is applied by adding j to the
+// exponent field.  x is clamped to >= -127, where f = 0, the polynomial is
+// exactly 1 and the exponent field becomes 0: the result is exactly +0.
+constexpr float EXP2_C1 = 0.6932829022407532f;
+constexpr float EXP2_C2 = 0.2422107607126236f;
+constexpr float EXP2_C3 = 0.055008746683597565f;
+constexpr float ROUND_MAGIC = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ uint64_t exp2_poly_pair(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  x0 = fmaxf(x0, -127.f);
+  x1 = fmaxf(x1, -127.f);
+  const uint64_t magic = f2_pack(ROUND_MAGIC, ROUND_MAGIC);
+  const uint64_t xc = f2_pack(x0, x1);
+  const uint64_t y = f2_add(xc, magic);          // j in the low mantissa bits
+  const uint64_t jf = f2_add(y, f2_pack(-ROUND_MAGIC, -ROUND_MAGIC));
+  const uint64_t f = f2_fma(jf, f2_pack(-1.f, -1.f), xc);  // exact: |x - j| <= 1/2
+  uint64_t pp = f2_fma(f2_pack(EXP2_C3, EXP2_C3), f, f2_pack(EXP2_C2, EXP2_C2));
+  pp = f2_fma(pp, f, f2_pack(EXP2_C1, EXP2_C1));
+  pp = f2_fma(pp, f, f2_pack(1.f, 1.f));
+  float p0, p1, y0, y1;
+  f2_unpack(pp, p0, p1);
+  f2_unpack(y, y0, y1);
+  // bits(y) << 23 == j << 23 (mod 2^32): the magic constant's low bits are 0.
+  const uint32_t r0 = __float_as_uint(p0) + (__float_as_uint(y0) << 23);
+  const uint32_t r1 = __float_as_uint(p1) + (__float_as_uint(y1) << 23);
+  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
+}
+}  // namespace ptx
+}  // namespace fa2
