@@ -84,7 +84,7 @@ static_assert(256 * REGS_SOFTMAX + 128 * REGS_CONTROL <= 384 * 168, "register sp
 // product build compiles every stamp away.
 #ifdef FA2_TRACE
 constexpr int TRACE_J = 64;   // K/V tiles recorded
-constexpr int TRACE_EV = 24;  // event kinds
+constexpr int TRACE_EV = 32;  // event kinds
 __device__ long long g_fa2_trace[TRACE_EV * TRACE_J + 1];
 #define FA2_STAMP(ev, j)                                                                          \
   do {                                                                                            \
@@ -143,6 +143,7 @@ struct Barriers {
   uint64_t p_full[2];   // softmax t wrote P_t(j) (and rescaled O_t if needed)
   uint64_t o_ready[2];  // last PV_t complete
   uint64_t mma_final[2];
+  uint64_t epi[2];      // the four warps of softmax group t wrote their O rows to shared memory
   uint32_t tmem_base;
   int abort;
 };
@@ -196,9 +197,9 @@ __device__ __forceinline__ int kv_tiles_for(int qb, int t, int n_kv_tiles) {
 // ------------------------------------------------------------------ softmax
 // One thread = one query row of tile t.  Returns false if a wait gave up.
 template <int HD, bool CAUSAL>
-__device__ __forceinline__ void softmax_role(const Params& p, Barriers* bars, volatile int* abort_flag,
-                                             uint32_t tmem, int t, int warp_in_wg, int lane, int row_g, int bh,
-                                             int n_t) {
+__device__ __forceinline__ void softmax_role(const Params& p, const CUtensorMap* tmap_o, uint32_t sQt, Barriers* bars,
+                                             volatile int* abort_flag, uint32_t tmem, int t, int warp_in_wg, int lane,
+                                             int row_g, int bh, int n_t) {
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp_in_wg * 32) << 16);
   const uint32_t s_addr = lane_base + tm_s(t);
   const uint32_t o_addr = lane_base + tm_o(t);
@@ -309,10 +310,14 @@ __device__ __forceinline__ void softmax_role(const Params& p, Barriers* bars, vo
   }
   if (ok) ok = wait_warp(smem_u32(&bars->o_ready[t]), 0, abort_flag, p.timeout_ns);
   if (!ok) return;
+  if (warp_in_wg == 0 && lane == 0) FA2_STAMP(24 + t, 0);
   tc_fence_after();
+  // Epilogue: O / l in bf16 is written into this tile's Q buffer (free: the
+  // o_ready commit tracks the tile's last S MMA) in the 128-byte-swizzled
+  // layout of the O tensor map, then one thread stores the tile with TMA.
   const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
   const bool store = row_g < p.N;
-  __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (store ? row_g : 0)) * HD;
+  const int r = warp_in_wg * 32 + lane;
   const uint64_t il = f2_pack(inv_l, inv_l);
 #pragma unroll
   for (int c = 0; c < HD / 32; ++c) {
@@ -327,22 +332,41 @@ __device__ __forceinline__ void softmax_role(const Params& p, Barriers* bars, vo
       f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), il), a0, a1);
       w[e] = pack_bf16x2(a0, a1);
     }
-    if (store) {
-      uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+    // 32 columns = 64 bytes = four 16-byte pieces of the row's 128-byte line
+    // in 64-column chunk c/2; piece k sits at (k ^ (r % 8)) * 16.
+    const uint32_t line = sQt + (c >> 1) * (128 * 128) + r * 128;
 #pragma unroll
-      for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+    for (int v = 0; v < 4; ++v) {
+      const int k = (c & 1) * 4 + v;
+      st_shared_v4(line + ((k ^ (r & 7)) << 4), w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
     }
+  }
+  // Every warp's rows are in shared memory before the store is issued; only
+  // the storing thread waits (bounded), so a warp that gave up earlier cannot
+  // leave the others blocked.
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(smem_u32(&bars->epi[t]));
+  const int tile_row0 = row_g - r;
+  if (warp_in_wg == 0 && lane == 0 && tile_row0 < p.N &&
+      wait_bounded(smem_u32(&bars->epi[t]), 0, abort_flag, p.timeout_ns, ROLE_SOFTMAX)) {
+#pragma unroll
+    for (int c = 0; c < HD / 64; ++c) tma_store_3d(tmap_o, sQt + c * (128 * 128), c * 64, tile_row0, bh);
+    bulk_commit_group();
+    bulk_wait_all();
   }
   if (store) {
     const float lse = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
     p.lse[static_cast<size_t>(bh) * p.N + row_g] = lse;
   }
+  if (warp_in_wg == 0 && lane == 0) FA2_STAMP(26 + t, 0);
 }
 
 template <int HD, bool CAUSAL>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const Params p) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
+                   const Params p) {
   using C = Cfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte-swizzle atoms.
@@ -382,6 +406,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     mbar_init(smem_u32(&bars->mma_final[0]), 1);
     mbar_init(smem_u32(&bars->mma_final[1]), 1);
+    mbar_init(smem_u32(&bars->epi[0]), 4);
+    mbar_init(smem_u32(&bars->epi[1]), 4);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -393,6 +419,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_out);
   }
   tc_fence_before();
   __syncthreads();
@@ -542,11 +569,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int warp_in_wg = warp & 3;    // TMEM lane quadrant
     const int r = warp_in_wg * 32 + lane;
     const int row_g = q0 + t * BM + r;
-    softmax_role<HD, CAUSAL>(p, bars, abort_flag, tmem, t, warp_in_wg, lane, row_g, bh, t == 0 ? n0 : n1);
+    softmax_role<HD, CAUSAL>(p, &tm_out, sQ + t * C::TILE_BYTES, bars, abort_flag, tmem, t, warp_in_wg, lane, row_g,
+                             bh, t == 0 ? n0 : n1);
   }
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) FA2_STAMP(28, 0);
   if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
@@ -639,8 +668,8 @@ static int validate(const void* q, const void* k, const void* v, const void* o, 
 }
 
 template <int HD, bool CAUSAL>
-static int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const Params& prm,
-                    int B, int H, cudaStream_t stream) {
+static int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                    const Params& prm, int B, int H, cudaStream_t stream) {
   using C = Cfg<HD>;
   auto kern = fa2_fwd_kernel<HD, CAUSAL>;
   static int attr_done_mask = 0;  // per device bit (devices 0..31)
@@ -658,7 +687,7 @@ static int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
     if (dev < 32) attr_done_mask |= (1 << dev);
   }
   dim3 grid(prm.n_q_blocks, H, B);
-  kern<<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, prm);
+  kern<<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_detail("kernel launch: %s", cudaGetErrorString(e));
@@ -672,11 +701,12 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   g_detail[0] = 0;
   int st = validate(q, k, v, o, lse, B, H, N, d, scale);
   if (st != FA2_OK) return st;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   const int BH = B * H;
   if ((st = make_tmap(&tq, q, d, N, BH)) != FA2_OK) return st;
   if ((st = make_tmap(&tk, k, d, N, BH)) != FA2_OK) return st;
   if ((st = make_tmap(&tv, v, d, N, BH)) != FA2_OK) return st;
+  if ((st = make_tmap(&to, o, d, N, BH)) != FA2_OK) return st;
   Params prm;
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
@@ -688,10 +718,10 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   prm.timeout_ns = timeout_ns;
   prm.inject_timeout = inject;
   if (d == 64)
-    return causal ? launch_t<64, true>(tq, tk, tv, prm, B, H, stream)
-                  : launch_t<64, false>(tq, tk, tv, prm, B, H, stream);
-  return causal ? launch_t<128, true>(tq, tk, tv, prm, B, H, stream)
-                : launch_t<128, false>(tq, tk, tv, prm, B, H, stream);
+    return causal ? launch_t<64, true>(tq, tk, tv, to, prm, B, H, stream)
+                  : launch_t<64, false>(tq, tk, tv, to, prm, B, H, stream);
+  return causal ? launch_t<128, true>(tq, tk, tv, to, prm, B, H, stream)
+                : launch_t<128, false>(tq, tk, tv, to, prm, B, H, stream);
 }
 
 constexpr unsigned long long DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s per wait
@@ -802,7 +832,7 @@ const char* fa2_last_error_detail(void) { return fa2::g_detail; }
 int fa2_version(void) { return 100; }
 
 #ifdef FA2_TRACE
-// Trace builds only: copy the timeline ((24 events x 64 tiles) + start) to host.
+// Trace builds only: copy the timeline ((32 events x 64 tiles) + start) to host.
 int fa2_trace_read(long long* host, int n) {
   if (!host || n < fa2::TRACE_EV * fa2::TRACE_J + 1) return FA2_ERR_INVALID_ARG;
   return cudaMemcpyFromSymbol(host, fa2::g_fa2_trace, sizeof(long long) * (fa2::TRACE_EV * fa2::TRACE_J + 1)) ==
