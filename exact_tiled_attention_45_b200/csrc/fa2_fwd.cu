@@ -73,10 +73,10 @@ constexpr float RESCALE_THRESHOLD = 8.0f;
 #define FA2_EMU_PAIRS_D64 3
 #endif
 // Register split: launched at 168 per thread (384 threads), the softmax
-// warpgroups grow to 216 and the control warpgroup shrinks to 64:
-// 256*216 + 128*64 = 63488 <= 384*168 = 64512.
+// warpgroups grow to 216 and the control warpgroup shrinks to 72:
+// 256*216 + 128*72 = 64512 <= 384*168 = 64512.
 constexpr uint32_t REGS_SOFTMAX = 216;
-constexpr uint32_t REGS_CONTROL = 64;
+constexpr uint32_t REGS_CONTROL = 72;
 static_assert(256 * REGS_SOFTMAX + 128 * REGS_CONTROL <= 384 * 168, "register split exceeds the launch budget");
 
 // Optional per-role timeline (compile with -DFA2_TRACE): SM clock stamps of
@@ -482,12 +482,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         wait_drain(smem_u32(&bars->v_full[t % C::VS]), (t / C::VS) & 1, p.timeout_ns);
     } else if (warp == MMA_WARP && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      // The tensor pipe keeps at most about one MMA queued, so the issuer does
-      // all of a step's waits first and then issues that step's MMAs back to
-      // back; every instruction between two MMAs is idle pipe time.
+      // The tensor pipe keeps about one MMA queued, so any wait or commit
+      // between two MMAs longer than one MMA (64 cycles) is idle pipe time.
+      // Only the softmax hand-offs are waited for between groups; the K/V
+      // waits run under the MMAs of the preceding group where possible.
       constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
-      auto issue_s = [&](int t, int ks) {
+      // `hook` runs after the second MMA of a group: a wait placed there
+      // overlaps the MMA the pipe is executing instead of idling it.
+      auto issue_s = [&](int t, int ks, auto&& hook) {
         const uint32_t qbase = sQ + t * C::TILE_BYTES;
         const uint32_t kbase = sK + ks * C::TILE_BYTES;
         const uint32_t d_s = tmem + tm_s(t);
@@ -496,63 +499,84 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
           mma_ss(d_s, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024), IDESC_S,
                  kk > 0 ? 1u : 0u);
+          if (kk == 1) hook();
         }
       };
-      auto issue_pv = [&](int t, int vs, bool acc) {
+      auto issue_pv = [&](int t, int vs, bool acc, auto&& hook) {
         const uint32_t vbase = sV + vs * C::TILE_BYTES;
         const uint32_t d_o = tmem + tm_o(t), a_p = tmem + tm_s(t);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
+        for (int kk = 0; kk < BN / 16; ++kk) {
           mma_ts(d_o, a_p + kk * 8, smem_desc_sw128(vbase + kk * 2048, C::CHUNK_BYTES, 1024), IDESC_PV,
                  (acc || kk > 0) ? 1u : 0u);
+          if (kk == 1) hook();
+        }
       };
       const unsigned long long to = p.timeout_ns;
+      bool ok = true;
       auto wait = [&](const uint64_t* bar, uint32_t parity) {
-        return wait_bounded(smem_u32(bar), parity, abort_flag, to, ROLE_MMA);
+        ok = ok && wait_bounded(smem_u32(bar), parity, abort_flag, to, ROLE_MMA);
       };
-      // K/V tile 0: S_0(0), S_1(0).
-      bool ok = wait(&bars->q_full[0], 0) && wait(&bars->k_full[0], 0);
+      auto nothing = [] {};
+      // K/V tile 0: S_0(0), S_1(0); Q_1 (and V_0 with a 3-stage V ring) are
+      // waited for under the MMAs.
+      wait(&bars->q_full[0], 0);
+      wait(&bars->k_full[0], 0);
       if (ok) {
         tc_fence_after();
-        issue_s(0, 0);
+        issue_s(0, 0, [&] { wait(&bars->q_full[1], 0); });
         mma_commit(smem_u32(&bars->s_full[0]));
         FA2_STAMP(3, 0);
-        ok = wait(&bars->q_full[1], 0);
       }
       if (ok) {
-        issue_s(1, 0);
+        issue_s(1, 0, [&] {
+          if (C::VS >= 3) wait(&bars->v_full[0], 0);
+        });
         mma_commit(smem_u32(&bars->s_full[1]));
         mma_commit(smem_u32(&bars->k_empty[0]));
         FA2_STAMP(7, 0);
       }
       // Step j: PV_0(j-1), S_0(j), PV_1(j-1), S_1(j).  Tile 0 may stop one
-      // K/V tile earlier (causal diagonal).
+      // K/V tile earlier (causal diagonal).  K(j) is waited for under PV_0's
+      // MMAs (PV_1's when tile 0 is done); with a 3-stage V ring V(j) is
+      // waited for under PV_1's MMAs of step j, otherwise at step j+1's start.
       for (int j = 1; ok && j <= n1; ++j) {
         const int i = j - 1;
         const int vs = i % C::VS;
         const int ks = j % C::KS;
         const bool do0 = i < n0, more0 = j < n0, more1 = j < n1;
+        auto wait_k = [&] {
+          if (more1) wait(&bars->k_full[ks], (j / C::KS) & 1);
+        };
         FA2_STAMP(0, i);
-        ok = (!do0 || wait(&bars->p_full[0], i & 1)) && wait(&bars->v_full[vs], (i / C::VS) & 1) &&
-             (!more1 || wait(&bars->k_full[ks], (j / C::KS) & 1));
-        if (!ok) break;
-        FA2_STAMP(1, i);
+        // V(j-1) from a 2-stage ring is waited for here, before the softmax
+        // hand-off (usually the later of the two), so its latency overlaps
+        // the softmax.
+        if (C::VS < 3) wait(&bars->v_full[vs], (i / C::VS) & 1);
         if (do0) {
+          wait(&bars->p_full[0], i & 1);
+          if (!ok) break;
+          FA2_STAMP(1, i);
           tc_fence_after();
-          issue_pv(0, vs, i > 0);
+          issue_pv(0, vs, i > 0, wait_k);
           FA2_STAMP(2, i);
-          if (more0) issue_s(0, ks);
+          if (!ok) break;
+          if (more0) issue_s(0, ks, nothing);
           mma_commit(smem_u32(more0 ? &bars->s_full[0] : &bars->o_ready[0]));
           FA2_STAMP(3, j);
         }
         FA2_STAMP(4, i);
-        ok = wait(&bars->p_full[1], i & 1);
+        wait(&bars->p_full[1], i & 1);
         if (!ok) break;
         FA2_STAMP(5, i);
         tc_fence_after();
-        issue_pv(1, vs, i > 0);
+        issue_pv(1, vs, i > 0, [&] {
+          if (!do0) wait_k();
+          if (C::VS >= 3 && more1) wait(&bars->v_full[j % C::VS], (j / C::VS) & 1);
+        });
         FA2_STAMP(6, i);
-        if (more1) issue_s(1, ks);
+        if (!ok) break;
+        if (more1) issue_s(1, ks, nothing);
         mma_commit(smem_u32(more1 ? &bars->s_full[1] : &bars->o_ready[1]));
         mma_commit(smem_u32(&bars->v_empty[vs]));
         if (more1) mma_commit(smem_u32(&bars->k_empty[ks]));
