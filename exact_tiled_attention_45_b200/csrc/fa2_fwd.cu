@@ -353,7 +353,7 @@ __device__ __forceinline__ void softmax_role(const Params& p, const CUtensorMap*
 #pragma unroll
     for (int c = 0; c < HD / 64; ++c) tma_store_3d(tmap_o, sQt + c * (128 * 128), c * 64, tile_row0, bh);
     bulk_commit_group();
-    bulk_wait_all();
+    bulk_wait_read();  // the shared-memory source must stay valid until read
   }
   if (store) {
     const float lse = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
