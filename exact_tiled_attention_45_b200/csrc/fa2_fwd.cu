@@ -319,17 +319,19 @@ __device__ __forceinline__ void softmax_role(const Params& p, const CUtensorMap*
   const bool store = row_g < p.N;
   const int r = warp_in_wg * 32 + lane;
   const uint64_t il = f2_pack(inv_l, inv_l);
+  uint32_t o[HD / 32][32];
+#pragma unroll
+  for (int c = 0; c < HD / 32; ++c) tmem_ld32(o_addr + c * 32, o[c]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < HD / 32; ++c) reg_fence32(o[c]);
 #pragma unroll
   for (int c = 0; c < HD / 32; ++c) {
-    uint32_t o[32];
-    tmem_ld32(o_addr + c * 32, o);
-    tmem_wait_ld();
-    reg_fence32(o);
     uint32_t w[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
       float a0, a1;
-      f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), il), a0, a1);
+      f2_unpack(f2_mul(f2_pack(__uint_as_float(o[c][2 * e]), __uint_as_float(o[c][2 * e + 1])), il), a0, a1);
       w[e] = pack_bf16x2(a0, a1);
     }
     // 32 columns = 64 bytes = four 16-byte pieces of the row's 128-byte line
