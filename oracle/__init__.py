@@ -3,4 +3,4 @@
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 legs import this package.  The CUDA path never does.
 """
-from .attention import attention_ref, attention_ref_rows, attention_probs  # noqa: F401
+from .attention import attention_probs, attention_ref, attention_ref_rect, attention_ref_rows  # noqa: F401

@@ -48,7 +48,7 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["attention_ref", "attention_ref_rows", "attention_probs"]
+__all__ = ["attention_ref", "attention_ref_rows", "attention_probs", "attention_ref_rect"]
 
 
 def _as_f64(x) -> np.ndarray:
@@ -58,21 +58,23 @@ def _as_f64(x) -> np.ndarray:
     return a
 
 
-def _allowed_mask(rows: np.ndarray, n_keys: int, causal: bool) -> np.ndarray:
+def _allowed_mask(rows: np.ndarray, n_keys: int, causal: bool, offset: int = 0) -> np.ndarray:
     """Boolean [len(rows), n_keys]: True where key j is allowed for query row i.
 
     Causal masking excludes keys after the query (iplexlaw blog, "Three changes
-    improve GPU utilisation" names causal-mask handling); with equal query and
-    key lengths that is j > i.
+    improve GPU utilisation" names causal-mask handling).  Query row i sits at
+    sequence position offset + i; with equal query and key lengths offset = 0
+    and the rule is j > i excluded.  With fewer queries than keys (decoding the
+    last Nq positions of an Nk-long sequence) offset = Nk - Nq.
     """
     j = np.arange(n_keys)[None, :]
     if causal:
-        return j <= rows[:, None]
+        return j <= rows[:, None] + offset
     return np.ones((rows.shape[0], n_keys), dtype=bool)
 
 
 def _rows_one_head(q_rows: np.ndarray, k: np.ndarray, v: np.ndarray,
-                   rows: np.ndarray, causal: bool, scale: float):
+                   rows: np.ndarray, causal: bool, scale: float, offset: int = 0):
     """Exact attention for selected query rows of one (batch, head).
 
     q_rows: [R, d] (the query vectors of ``rows``), k, v: [N, d].
@@ -82,7 +84,7 @@ def _rows_one_head(q_rows: np.ndarray, k: np.ndarray, v: np.ndarray,
     # Scores: the full R x N block, materialised (the "standard attention"
     # the abstract contrasts with the tiled method).
     s = scale * (q_rows @ k.T)
-    allowed = _allowed_mask(rows, n_keys, causal)
+    allowed = _allowed_mask(rows, n_keys, causal, offset)
     s = np.where(allowed, s, -np.inf)
     m = np.max(s, axis=1, keepdims=True)                 # row max over allowed keys
     empty = ~np.isfinite(m)                              # row with no allowed key
@@ -162,3 +164,33 @@ def attention_probs(q, k, causal: bool = False, scale: float | None = None):
             e = np.exp(s - m)
             p[b, h] = e / np.sum(e, axis=1, keepdims=True)
     return p
+
+
+def attention_ref_rect(q, k, v, causal: bool = False, scale: float | None = None,
+                       row_block: int = 2048):
+    """Exact attention with Nq query rows and Nk >= Nq keys.
+
+    q: [B, H, Nq, d]; k, v: [B, H, Nk, d].  Query row i is sequence position
+    Nk - Nq + i (the last Nq positions, as when decoding or prefilling a
+    chunk after a cached prefix); causal masking excludes keys after that
+    position.  With Nq == Nk this is exactly :func:`attention_ref`.
+    Returns (O [B, H, Nq, d], LSE [B, H, Nq]) in float64.
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if k.shape != (B, H, Nk, d) or v.shape != (B, H, Nk, d) or Nq > Nk:
+        raise ValueError("need q [B,H,Nq,d], k and v [B,H,Nk,d] with Nq <= Nk")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    offset = Nk - Nq
+    o = np.empty((B, H, Nq, d), dtype=np.float64)
+    lse = np.empty((B, H, Nq), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            for r0 in range(0, Nq, row_block):
+                rows = np.arange(r0, min(Nq, r0 + row_block))
+                ob, lb = _rows_one_head(q[b, h, rows], k[b, h], v[b, h], rows, causal, float(scale), offset)
+                o[b, h, rows] = ob
+                lse[b, h, rows] = lb
+    return o, lse

@@ -312,14 +312,14 @@ def test_bf16_inputs_taken_exactly():
 # Mutation test: plausible mistakes planted in the oracle fail a pin
 # --------------------------------------------------------------------------
 
-def _flipped_mask(rows, n_keys, causal):
+def _flipped_mask(rows, n_keys, causal, offset=0):
     j = np.arange(n_keys)[None, :]
-    return (j >= rows[:, None]) if causal else np.ones((rows.shape[0], n_keys), bool)
+    return (j >= rows[:, None] + offset) if causal else np.ones((rows.shape[0], n_keys), bool)
 
 
-def _strict_mask(rows, n_keys, causal):
+def _strict_mask(rows, n_keys, causal, offset=0):
     j = np.arange(n_keys)[None, :]
-    return (j < rows[:, None]) if causal else np.ones((rows.shape[0], n_keys), bool)
+    return (j < rows[:, None] + offset) if causal else np.ones((rows.shape[0], n_keys), bool)
 
 
 def _make_rows(bug, block=4):
