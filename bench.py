@@ -15,6 +15,11 @@ value is the FLOPs of all ranks divided by the slowest rank's time.
 
 ``--impl reference`` times the fp64 CPU oracle on this host's cores instead,
 each step on a bounded sample of heads of the same workload (rank 0 only).
+
+Decode workloads (``--workload decode_...`` / ``chunk_...``: Nq queries at the
+end of an Nk-long sequence) run the split-K/V entry point instead; a step is
+one call (range kernel + merge kernel) and the metric is effective HBM GB/s:
+the bytes of Q, K, V read once and O, LSE written once, over the step time.
 """
 from __future__ import annotations
 
@@ -34,7 +39,9 @@ METRIC = "attn fwd TFLOP/s (bf16, N=512–16k, d=64/128) and % of B200 dense BF1
 DEFAULT_WORKLOAD = "B8_H16_N2048_d128_causal"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_BF16_TFLOPS = 2250.0
-KERNEL_SOURCES = ["exact_tiled_attention_45_b200/csrc/fa2_fwd.cu", "exact_tiled_attention_45_b200/csrc/sm100_ptx.cuh"]
+DECODE_METRIC = "split-K/V attn fwd effective HBM GB/s (Q,K,V read once, O,LSE written once)"
+KERNEL_SOURCES = ["exact_tiled_attention_45_b200/csrc/fa2_fwd.cu", "exact_tiled_attention_45_b200/csrc/sm100_ptx.cuh",
+                  "exact_tiled_attention_45_b200/csrc/fa2_splitkv.cuh"]
 
 
 def parse_args():
@@ -47,6 +54,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the timed oracle sample")
+    ap.add_argument("--splits", type=int, default=0, help="key ranges for decode workloads (0 = library choice)")
     return ap.parse_args()
 
 
@@ -191,23 +199,43 @@ def cpu_oracle_sample(w, budget_s: float, q, k, v):
             "seconds": round(dt, 2)}, np
 
 
+def is_decode(w) -> bool:
+    return hasattr(w, "Nq")
+
+
+def oracle_head(w, q, k, v, b, h):
+    """The fp64 oracle on head (b, h) of the workload."""
+    from oracle import attention_ref, attention_ref_rect
+    fn = attention_ref_rect if is_decode(w) else attention_ref
+    return fn(q[b:b + 1, h:h + 1].double().numpy(), k[b:b + 1, h:h + 1].double().numpy(),
+              v[b:b + 1, h:h + 1].double().numpy(), causal=w.causal, scale=w.d ** -0.5)
+
+
+def workload_inputs(w, seed):
+    from exact_tiled_attention_45_b200.inputs import make_q_kv, make_qkv
+    if is_decode(w):
+        return make_q_kv(w.B, w.H, w.Nq, w.Nk, w.d, seed=seed, qk_mult=w.qk_mult)
+    return make_qkv(w.B, w.H, w.N, w.d, seed=seed, qk_mult=w.qk_mult)
+
+
 def run_reference(args, w):
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
     import torch
-    from exact_tiled_attention_45_b200.inputs import make_qkv
-    from oracle import attention_ref
     heads_per_step = 1
-    q, k, v = make_qkv(w.B, w.H, w.N, w.d, seed=0, qk_mult=w.qk_mult)
+    q, k, v = workload_inputs(w, 0)
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
-    per_head = w.flops / (w.B * w.H)
+    if is_decode(w):
+        per_head, unit, metric, scale_u = w.bytes / (w.B * w.H), "GB/s", DECODE_METRIC, 1e9
+        heads_per_step = 16
+    else:
+        per_head, unit, metric, scale_u = w.flops / (w.B * w.H), "TFLOP/s", METRIC, 1e12
 
     def step(i):
         for t in range(heads_per_step):
             b, h = heads[(i * heads_per_step + t) % len(heads)]
-            attention_ref(q[b:b + 1, h:h + 1].double().numpy(), k[b:b + 1, h:h + 1].double().numpy(),
-                          v[b:b + 1, h:h + 1].double().numpy(), causal=w.causal, scale=w.d ** -0.5)
+            oracle_head(w, q, k, v, b, h)
 
     for i in range(args.warmup):
         step(i)
@@ -215,16 +243,163 @@ def run_reference(args, w):
     for i in range(args.steps):
         step(args.warmup + i)
     dt = time.perf_counter() - t0
-    value = per_head * heads_per_step * args.steps / dt / 1e12
+    value = per_head * heads_per_step * args.steps / dt / scale_u
     cores = torch.get_num_threads()
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": dict(w.as_dict(), sample=f"{heads_per_step} head(s) of {w.B * w.H} per step"),
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": int(cores), "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": unit, "cores": int(cores), "kind": "oracle",
                          "sample": f"{heads_per_step} head(s) per step of {w.name}, fp64 NumPy on host cores"},
-        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_decode(args, w):
+    """Split-K/V entry point on a decode workload; effective HBM GB/s."""
+    import torch
+    import torch.distributed as dist
+    import exact_tiled_attention_45_b200 as fa2
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    q_h, k_h, v_h = workload_inputs(w, shard_seed(rank))
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    splits = fa2.splitkv_splits(w.B, w.H, w.Nq, w.Nk, w.d, args.splits)
+    ws_bytes = fa2.splitkv_workspace_bytes(w.B, w.H, w.Nq, w.Nk, w.d, args.splits)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+    in_bytes = (q.numel() + k.numel() + v.numel()) * 2
+    out_bytes = o.numel() * 2 + lse.numel() * 4
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev) if in_bytes <= l2_bytes else None
+
+    def call():
+        fa2.fwd_splitkv(q, k, v, causal=w.causal, n_splits=args.splits, out=o, lse=lse, workspace=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.zero_()
+        call()
+    fa2.sync_status(stream)
+    sampler = ClockSampler(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    if flush is None:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            call()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        total_ms = ev0.elapsed_time(ev1)
+    else:
+        total_ms = 0.0
+        for _ in range(args.steps):
+            flush.zero_()
+            ev0.record(stream)
+            call()
+            ev1.record(stream)
+            ev1.synchronize()
+            total_ms += ev0.elapsed_time(ev1)
+    sampler.stop()
+    barrier()
+    fa2.sync_status(stream)
+    step_ms = total_ms / args.steps
+    max_ms = max_over_ranks(total_ms, dev) / args.steps
+    value = w.bytes * world / (max_ms * 1e-3) / 1e9
+
+    # End to end: pinned host Q, K, V copied in, the call, O and LSE copied
+    # back, all on the stream inside the timed region.
+    e2e = None
+    if not args.no_e2e:
+        qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+        op = torch.empty_like(qp).pin_memory()
+        lp = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32).pin_memory()
+        e2e_steps = max(3, min(args.steps, 10))
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                q.copy_(qp, non_blocking=True)
+                k.copy_(kp, non_blocking=True)
+                v.copy_(vp, non_blocking=True)
+                call()
+                op.copy_(o, non_blocking=True)
+                lp.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), dev) / e2e_steps
+        e2e = {"value": w.bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes, "steps": e2e_steps,
+               "path": "torch pinned copies + fwd_splitkv on one stream"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    # A long chunk of queries is a contraction again: above the ridge point
+    # (FLOP per byte = peak FLOP/s / peak B/s) the tensor roofline applies.
+    if w.flops / w.bytes > tf * 1e12 / (hbm * 1e9):
+        roof = {"bound": "tensor", "achieved": w.flops / (step_ms * 1e-3) / 1e12, "peak": tf, "unit": "TFLOP/s",
+                "peak_source": f"{peak_kind} bf16 burst"}
+    else:
+        roof = {"bound": "hbm", "achieved": w.bytes / (step_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                "peak_source": f"{peak_kind} copy bandwidth"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        import numpy as np  # noqa: F401
+        heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+        done, t0 = 0, time.perf_counter()
+        for b, h in heads:
+            oracle_head(w, q_h, k_h, v_h, b, h)
+            done += 1
+            if time.perf_counter() - t0 >= args.cpu_seconds:
+                break
+        dt = time.perf_counter() - t0
+        cpu = {"value": w.bytes / (w.B * w.H) * done / dt / 1e9, "unit": "GB/s", "cores": torch.get_num_threads(),
+               "kind": "oracle", "sample": f"{done} of {len(heads)} heads of {w.name} (fp64 NumPy, {dt:.1f} s)"}
+    line = {
+        "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(w.as_dict(), seed="rank", scale=f"1/sqrt({w.d})", n_splits=splits,
+                       l2=("inputs larger than L2" if flush is None else "L2 flushed before every step"),
+                       parallelism=("single GPU" if world == 1 else f"{world} ranks, independent heads, no collective")),
+        "tflops": w.flops / (step_ms * 1e-3) / 1e12,
+        "roofline": dict(roof, traffic=recorded_traffic(w.name, source_hash()),
+                         kernel=("fa2_splitkv_kernel (one range, no merge)" if splits == 1 else
+                                 "fa2_splitkv_kernel + fa2_splitkv_combine_kernel (one step, both timed)"),
+                         src=source_hash()),
+        "clocks": sampler.summary(),
+        "gpu_launches": (1 if splits == 1 else 2) * args.steps,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -238,6 +413,10 @@ def main():
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.steps < 1 or args.warmup < 3:
+        raise SystemExit("need --steps >= 1 and --warmup >= 3")
+    if is_decode(w):
+        return run_decode(args, w)
 
     import torch
     import torch.distributed as dist

@@ -21,7 +21,8 @@ FA2_OK, FA2_ERR_INVALID_ARG, FA2_ERR_UNSUPPORTED, FA2_ERR_CUDA, FA2_ERR_TIMEOUT 
 
 #: Every symbol the header declares.
 EXPORTS = ("fa2_fwd", "fa2_fwd_host", "fa2_fwd_host_workspace_bytes", "fa2_sync_status",
-           "fa2_fwd_inject_timeout", "fa2_strerror", "fa2_last_error_detail", "fa2_version")
+           "fa2_fwd_inject_timeout", "fa2_fwd_splitkv", "fa2_fwd_splitkv_splits",
+           "fa2_fwd_splitkv_workspace_bytes", "fa2_strerror", "fa2_last_error_detail", "fa2_version")
 
 _lib = None
 
@@ -47,6 +48,13 @@ def load() -> ctypes.CDLL:
     lib.fa2_sync_status.restype = _int
     lib.fa2_fwd_inject_timeout.argtypes = _FWD_ARGS + [ctypes.c_ulonglong, _vp]
     lib.fa2_fwd_inject_timeout.restype = _int
+    lib.fa2_fwd_splitkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _float, _int, _vp,
+                                    ctypes.c_size_t, _vp]
+    lib.fa2_fwd_splitkv.restype = _int
+    lib.fa2_fwd_splitkv_splits.argtypes = [_int] * 6
+    lib.fa2_fwd_splitkv_splits.restype = _int
+    lib.fa2_fwd_splitkv_workspace_bytes.argtypes = [_int] * 6
+    lib.fa2_fwd_splitkv_workspace_bytes.restype = ctypes.c_size_t
     lib.fa2_strerror.argtypes = [_int]
     lib.fa2_strerror.restype = ctypes.c_char_p
     lib.fa2_last_error_detail.argtypes = []
@@ -168,3 +176,62 @@ def fwd_inject_timeout(q, k, v, causal=False, scale=None, timeout_ns: int = 50_0
                                     B, H, N, d, int(bool(causal)), float(scale), int(timeout_ns), h)
     _check(st, lib)
     return lib.fa2_sync_status(h)
+
+
+def _check_q_kv(q, k, v):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be 4-D, got {tuple(t.shape)}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.device.type != "cuda":
+            raise ValueError(f"{name} must be on cuda, got {t.device}")
+    B, H, Nq, d = q.shape
+    if k.shape != v.shape or k.shape[0] != B or k.shape[1] != H or k.shape[3] != d:
+        raise ValueError("need q [B, H, Nq, d] and k, v [B, H, Nk, d]")
+    if Nq > k.shape[2]:
+        raise ValueError("need Nq <= Nk")
+
+
+def splitkv_splits(B: int, H: int, Nq: int, Nk: int, d: int, n_splits: int = 0) -> int:
+    """Number of key ranges fwd_splitkv uses for this shape (0 on bad sizes)."""
+    return int(load().fa2_fwd_splitkv_splits(B, H, Nq, Nk, d, n_splits))
+
+
+def splitkv_workspace_bytes(B: int, H: int, Nq: int, Nk: int, d: int, n_splits: int = 0) -> int:
+    return int(load().fa2_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, n_splits))
+
+
+def fwd_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+                scale: float | None = None, n_splits: int = 0, out: torch.Tensor | None = None,
+                lse: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """Exact attention of Nq queries (the last Nq positions) against Nk >= Nq keys.
+
+    q: [B, H, Nq, d]; k, v: [B, H, Nk, d] (bf16, CUDA, contiguous).  The keys
+    are split into ``n_splits`` ranges (0 = chosen by the library) processed
+    by separate CTAs, then merged.  ``workspace`` is an optional uint8 CUDA
+    tensor of at least :func:`splitkv_workspace_bytes` bytes, 256-byte aligned
+    (none is needed, and the merge is skipped, when one range is used).
+    Returns (O bf16 [B, H, Nq, d], LSE fp32 [B, H, Nq]).
+    """
+    lib = load()
+    _check_q_kv(q, k, v)
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = splitkv_workspace_bytes(B, H, Nq, Nk, d, n_splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr, ws_len = (workspace.data_ptr(), workspace.numel()) if workspace is not None else (None, 0)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    st = lib.fa2_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                             B, H, Nq, Nk, d, int(bool(causal)), float(scale), int(n_splits),
+                             ws_ptr, ws_len, _stream_handle(stream))
+    _check(st, lib)
+    return out, lse

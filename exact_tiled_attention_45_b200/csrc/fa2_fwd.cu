@@ -40,6 +40,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdint>
@@ -608,6 +609,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+#include "fa2_splitkv.cuh"
+
 // ====================================================================== host
 
 static thread_local char g_detail[512] = "";
@@ -668,8 +671,8 @@ static int validate(const void* q, const void* k, const void* v, const void* o, 
     set_detail("bad sizes B=%d H=%d N=%d", B, H, N);
     return FA2_ERR_INVALID_ARG;
   }
-  if (!std::isfinite(scale)) {
-    set_detail("scale is not finite");
+  if (!std::isfinite(scale) || !(scale > 0.f)) {
+    set_detail("scale must be finite and positive");
     return FA2_ERR_INVALID_ARG;
   }
   if (d != 64 && d != 128) {
@@ -751,6 +754,164 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
 }
 
 constexpr unsigned long long DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s per wait
+
+// ------------------------------------------------------------------ split-K/V host side
+
+constexpr int SKV_MAX_SPLITS = 128;
+
+static int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) ==
+                                                 cudaSuccess && n > 0)
+    return n;
+  cudaGetLastError();  // no device here: plan for a B200
+  return 148;
+}
+
+static bool skv_sizes_ok(int B, int H, int Nq, int Nk) {
+  return B >= 1 && H >= 1 && Nq >= 1 && Nk >= Nq && static_cast<long long>(B) * H <= 65535;
+}
+
+// Number of key ranges actually used.  n_splits = 0 picks one: the work is a
+// stream over K and V, so what matters is enough CTAs to keep most SMs
+// loading; beyond that each extra range only adds set-up, partial writes and
+// the merge.  So: the fewest ranges that give at least 0.8 x (SM count) CTAs,
+// keeping at least 4 key tiles per range.  A requested count is capped at 128
+// and at the number of key tiles, then reduced to ceil(tiles / ceil(tiles /
+// s)) so that no range is empty by construction.
+static int skv_resolve_splits(int B, int H, int Nq, int Nk, int n_splits) {
+  const int n_kv = (Nk + BN - 1) / BN;
+  int s = n_splits;
+  if (s <= 0) {
+    const long long base = static_cast<long long>((Nq + BM - 1) / BM) * B * H;
+    const long long want = (static_cast<long long>(sm_count()) * 4 + 4) / 5;
+    s = base >= want ? 1 : static_cast<int>((want + base - 1) / base);
+    s = std::max(1, std::min(s, n_kv / 4));
+  }
+  s = std::min(std::min(s, SKV_MAX_SPLITS), n_kv);
+  const int tps = (n_kv + s - 1) / s;
+  return (n_kv + tps - 1) / tps;
+}
+
+static size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace layout: o_part fp32 [splits, B*H, Nq, d], then lse_part fp32
+// [splits, B*H, Nq], each starting on a 256-byte boundary.  A single range
+// needs none.
+static size_t skv_workspace_bytes(int B, int H, int Nq, int d, int splits) {
+  if (splits <= 1) return 0;
+  const size_t rows = static_cast<size_t>(splits) * B * H * Nq;
+  return round256(rows * d * 4) + round256(rows * 4);
+}
+
+template <int HD, bool CAUSAL>
+static int skv_launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const SkvParams& prm,
+                        int n_q_tiles, int splits, __nv_bfloat16* o, float* lse, cudaStream_t stream) {
+  using C = SkvCfg<HD>;
+  auto kern = fa2_splitkv_kernel<HD, CAUSAL>;
+  static int attr_done_mask = 0;  // per device bit (devices 0..31)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    set_detail("cudaGetDevice failed");
+    return FA2_ERR_CUDA;
+  }
+  if (dev >= 32 || !(attr_done_mask & (1 << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) {
+      set_detail("cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+      return FA2_ERR_CUDA;
+    }
+    if (dev < 32) attr_done_mask |= (1 << dev);
+  }
+  kern<<<dim3(n_q_tiles, prm.BH, splits), SKV_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_detail("split-K/V kernel launch: %s", cudaGetErrorString(e));
+    return FA2_ERR_CUDA;
+  }
+  if (prm.direct) return FA2_OK;
+  const int rows = prm.BH * prm.Nq;
+  fa2_splitkv_combine_kernel<HD><<<(rows + 3) / 4, 128, 0, stream>>>(prm.o_part, prm.lse_part, o, lse, rows, splits);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_detail("merge kernel launch: %s", cudaGetErrorString(e));
+    return FA2_ERR_CUDA;
+  }
+  return FA2_OK;
+}
+
+static int splitkv_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                        int Nk, int d, int causal, float scale, int n_splits, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream) {
+  g_detail[0] = 0;
+  if (!q || !k || !v || !o || !lse) {
+    set_detail("null pointer");
+    return FA2_ERR_INVALID_ARG;
+  }
+  if (!skv_sizes_ok(B, H, Nq, Nk) || n_splits < 0) {
+    set_detail("bad sizes B=%d H=%d Nq=%d Nk=%d n_splits=%d (need Nq >= 1, Nk >= Nq, B*H <= 65535)", B, H, Nq,
+               Nk, n_splits);
+    return FA2_ERR_INVALID_ARG;
+  }
+  if (!std::isfinite(scale) || !(scale > 0.f)) {
+    set_detail("scale must be finite and positive");
+    return FA2_ERR_INVALID_ARG;
+  }
+  if (d != 64 && d != 128) {
+    set_detail("head dimension %d not supported (64 or 128)", d);
+    return FA2_ERR_UNSUPPORTED;
+  }
+  const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                        reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o);
+  if ((mis & 15u) || (reinterpret_cast<uintptr_t>(lse) & 3u)) {
+    set_detail("misaligned pointer (q/k/v/o need 16 bytes, lse 4)");
+    return FA2_ERR_INVALID_ARG;
+  }
+  const int splits = skv_resolve_splits(B, H, Nq, Nk, n_splits);
+  const size_t need = skv_workspace_bytes(B, H, Nq, d, splits);
+  if (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)) {
+    set_detail("workspace missing, misaligned or too small: %zu bytes, need %zu (256-byte aligned) for %d key ranges",
+               workspace_bytes, need, splits);
+    return FA2_ERR_INVALID_ARG;
+  }
+  const size_t BH = static_cast<size_t>(B) * H;
+  const size_t qb = BH * Nq * d * 2, kb = BH * Nk * d * 2, lb = BH * Nq * 4;
+  if (overlap(o, qb, q, qb) || overlap(o, qb, k, kb) || overlap(o, qb, v, kb) || overlap(o, qb, lse, lb) ||
+      overlap(lse, lb, q, qb) || overlap(lse, lb, k, kb) || overlap(lse, lb, v, kb) ||
+      (need > 0 && (overlap(workspace, need, q, qb) || overlap(workspace, need, k, kb) ||
+                    overlap(workspace, need, v, kb) || overlap(workspace, need, o, qb) ||
+                    overlap(workspace, need, lse, lb)))) {
+    set_detail("output or workspace buffers overlap inputs or each other");
+    return FA2_ERR_INVALID_ARG;
+  }
+  CUtensorMap tq, tk, tv;
+  int st;
+  if ((st = make_tmap(&tq, q, d, Nq, static_cast<int>(BH))) != FA2_OK) return st;
+  if ((st = make_tmap(&tk, k, d, Nk, static_cast<int>(BH))) != FA2_OK) return st;
+  if ((st = make_tmap(&tv, v, d, Nk, static_cast<int>(BH))) != FA2_OK) return st;
+  SkvParams prm;
+  prm.direct = splits == 1;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.o_part = prm.direct ? nullptr : static_cast<float*>(workspace);
+  prm.lse_part = prm.direct ? nullptr
+                            : reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                                       round256(static_cast<size_t>(splits) * BH * Nq * d * 4));
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.BH = static_cast<int>(BH);
+  prm.n_kv_tiles = (Nk + BN - 1) / BN;
+  prm.tiles_per_split = (prm.n_kv_tiles + splits - 1) / splits;
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+  prm.timeout_ns = DEFAULT_TIMEOUT_NS;
+  const int n_q_tiles = (Nq + BM - 1) / BM;
+  auto* ob = static_cast<__nv_bfloat16*>(o);
+  if (d == 64)
+    return causal ? skv_launch_t<64, true>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
+                  : skv_launch_t<64, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
+  return causal ? skv_launch_t<128, true>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
+                : skv_launch_t<128, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
+}
 
 }  // namespace fa2
 
@@ -840,6 +1001,24 @@ int fa2_fwd_host(const void* q, const void* k, const void* v, void* o, float* ls
     return FA2_ERR_CUDA;
   }
   return fa2_sync_status(stream);
+}
+
+int fa2_fwd_splitkv_splits(int B, int H, int Nq, int Nk, int d, int n_splits) {
+  if (!fa2::skv_sizes_ok(B, H, Nq, Nk) || n_splits < 0 || (d != 64 && d != 128)) return 0;
+  return fa2::skv_resolve_splits(B, H, Nq, Nk, n_splits);
+}
+
+size_t fa2_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int n_splits) {
+  const int splits = fa2_fwd_splitkv_splits(B, H, Nq, Nk, d, n_splits);
+  if (splits == 0) return 0;
+  return fa2::skv_workspace_bytes(B, H, Nq, d, splits);
+}
+
+int fa2_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                    int d, int causal, float scale, int n_splits, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  return fa2::splitkv_impl(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, n_splits, workspace, workspace_bytes,
+                           static_cast<cudaStream_t>(stream));
 }
 
 const char* fa2_strerror(int status) {

@@ -1,0 +1,445 @@
+// Split-K/V exact attention for few queries against many keys (decoding, or a
+// prefill chunk after a cached prefix).  Included by fa2_fwd.cu inside
+// namespace fa2 (one translation unit: shares the status word and helpers).
+//
+// The pages distinguish the initial processing of a long prompt from
+// token-by-token generation, whose bottlenecks differ (iplexlaw blog
+// "FlashAttention-2: making long-context attention run efficiently on GPUs",
+// section "Document the implementation difference").  With few query rows the
+// work is a stream over K and V (HBM-bound), and one query block per head
+// leaves most SMs idle; so the keys are split into ranges processed by
+// separate CTAs, each producing a partial result normalised over its own range
+// with that range's logsumexp, and a second kernel merges them exactly:
+//     LSE = ln sum_s exp(LSE_s),   O = sum_s exp(LSE_s - LSE) O_s.
+// Query row i sits at sequence position Nk - Nq + i (the last Nq positions);
+// causal masking excludes keys after that position.
+//
+// With a single range the partial kernel writes the final bf16 O and LSE
+// itself and no merge runs.
+//
+// Partial kernel: one CTA per (128-row query tile, batch*head, key range);
+// 192 threads: warps 0-3 softmax (thread r <-> row r <-> TMEM lane r), warp 4
+// TMA producer, warp 5 MMA issuer.  TMEM: two score buffers (the next S is
+// computed while the softmax works on the current one), a separate P buffer,
+// and O.  Rows past Nq are computed on zero queries and never stored.
+
+constexpr int SKV_THREADS = 192;
+constexpr int SKV_PRODUCER_WARP = 4;
+constexpr int SKV_MMA_WARP = 5;
+constexpr uint32_t SKV_TM_S0 = 0, SKV_TM_S1 = 128, SKV_TM_P = 256, SKV_TM_O = 384;
+
+template <int HD>
+struct SkvCfg {
+  static constexpr int KCH = HD / 64;
+  static constexpr int CHUNK_BYTES = 128 * 128;
+  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;
+  // Deep K/V rings: the stream over keys is the bound, so keep many tiles in
+  // flight (224 KB of rings for d = 128, 128 KB for d = 64).
+  static constexpr int KS = (HD == 128) ? 3 : 4;
+  static constexpr int VS = KS;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VS * TILE_BYTES;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct SkvParams {
+  float* o_part;    // [n_splits, B*H, Nq, d] fp32, normalised within the range
+  float* lse_part;  // [n_splits, B*H, Nq] fp32 natural-log logsumexp of the range
+  __nv_bfloat16* o; // final outputs, written directly when there is one range
+  float* lse;
+  int direct;       // 1: one range, no merge step
+  int Nq;
+  int Nk;
+  int BH;
+  int n_kv_tiles;       // ceil(Nk / 128)
+  int tiles_per_split;  // key tiles per range
+  float scale_log2;
+  unsigned long long timeout_ns;
+};
+
+struct SkvBarriers {
+  uint64_t q_full;
+  uint64_t k_full[4], k_empty[4];
+  uint64_t v_full[4], v_empty[4];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full;
+  uint64_t pv_done;
+  uint64_t mma_final;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(SkvBarriers) <= 256, "barrier block");
+
+template <int HD, bool CAUSAL>
+__global__ void __launch_bounds__(SKV_THREADS, 1)
+    fa2_splitkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const SkvParams p) {
+  using C = SkvCfg<HD>;
+  const int q_first = static_cast<int>(blockIdx.x) * BM;
+  const int bh = static_cast<int>(blockIdx.y);
+  const int split = static_cast<int>(blockIdx.z);
+  const int offset = p.Nk - p.Nq;  // sequence position of query row 0
+  // Key tiles this query tile needs: all of them, or (causal) up to the
+  // position of its last row.
+  int n_need = p.n_kv_tiles;
+  if (CAUSAL) n_need = min(n_need, (offset + min(q_first + BM, p.Nq) - 1) / BN + 1);
+  const int kt_begin = split * p.tiles_per_split;
+  const int kt_end = min(kt_begin + p.tiles_per_split, n_need);
+  const int nkv = kt_end - kt_begin;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (nkv <= 0) {
+    // Nothing of this range is visible to this tile: an empty partial.
+    if (warp < 4) {
+      const int row = q_first + warp * 32 + lane;
+      if (row < p.Nq) {
+        const size_t prow = (static_cast<size_t>(split) * p.BH + bh) * p.Nq + row;
+        p.lse_part[prow] = -INFINITY;
+        float4* dst = reinterpret_cast<float4*>(p.o_part + prow * HD);
+#pragma unroll
+        for (int c = 0; c < HD / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    return;
+  }
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+  SkvBarriers* bars = reinterpret_cast<SkvBarriers*>(smem + C::OFF_BAR);
+  volatile int* abort_flag = &bars->abort;
+  const uint32_t sQ = base + C::OFF_Q;
+  const uint32_t sK = base + C::OFF_K;
+  const uint32_t sV = base + C::OFF_V;
+  const uint32_t b_q = smem_u32(&bars->q_full);
+  const uint32_t b_p = smem_u32(&bars->p_full);
+  const uint32_t b_pv = smem_u32(&bars->pv_done);
+  const uint32_t b_final = smem_u32(&bars->mma_final);
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_q, 1);
+    for (int s = 0; s < C::KS; ++s) {
+      mbar_init(smem_u32(&bars->k_full[s]), 1);
+      mbar_init(smem_u32(&bars->k_empty[s]), 1);
+    }
+    for (int s = 0; s < C::VS; ++s) {
+      mbar_init(smem_u32(&bars->v_full[s]), 1);
+      mbar_init(smem_u32(&bars->v_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&bars->s_full[s]), 1);
+      mbar_init(smem_u32(&bars->s_free[s]), 4);
+    }
+    mbar_init(b_p, 4);
+    mbar_init(b_pv, 1);
+    mbar_init(b_final, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == SKV_MMA_WARP) {
+    tmem_alloc(smem_u32(&bars->tmem_base), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == SKV_PRODUCER_WARP && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const unsigned long long to = p.timeout_ns;
+
+  if (warp == SKV_PRODUCER_WARP) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(b_q, C::TILE_BYTES);
+      for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * C::CHUNK_BYTES, &tm_q, b_q, c * 64, q_first, bh);
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < nkv; ++j) {
+        const int kv0 = (kt_begin + j) * BN;
+        const int ks = j % C::KS;
+        if (j >= C::KS &&
+            !wait_bounded(smem_u32(&bars->k_empty[ks]), ((j / C::KS) - 1) & 1, abort_flag, to, ROLE_PRODUCER))
+          break;
+        const uint32_t kb = smem_u32(&bars->k_full[ks]);
+        mbar_arrive_expect_tx(kb, C::TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sK + ks * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_k, kb, c * 64, kv0, bh);
+        ++k_issued;
+        const int vs = j % C::VS;
+        if (j >= C::VS &&
+            !wait_bounded(smem_u32(&bars->v_empty[vs]), ((j / C::VS) - 1) & 1, abort_flag, to, ROLE_PRODUCER))
+          break;
+        const uint32_t vb = smem_u32(&bars->v_full[vs]);
+        mbar_arrive_expect_tx(vb, C::TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sV + vs * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_v, vb, c * 64, kv0, bh);
+        ++v_issued;
+      }
+      wait_drain(b_q, 0, to);
+      for (int x = (k_issued > C::KS ? k_issued - C::KS : 0); x < k_issued; ++x)
+        wait_drain(smem_u32(&bars->k_full[x % C::KS]), (x / C::KS) & 1, to);
+      for (int x = (v_issued > C::VS ? v_issued - C::VS : 0); x < v_issued; ++x)
+        wait_drain(smem_u32(&bars->v_full[x % C::VS]), (x / C::VS) & 1, to);
+    }
+  } else if (warp == SKV_MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    // Order S(0), S(1), PV(0), S(2), PV(1), ...: the next scores are computed
+    // while the softmax works on the current ones.
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
+      bool ok = wait_bounded(b_q, 0, abort_flag, to, ROLE_MMA);
+      for (int j = 0; ok && j <= nkv; ++j) {
+        if (j < nkv) {
+          const int ks = j % C::KS;
+          const int sb = j & 1;
+          if (!wait_bounded(smem_u32(&bars->k_full[ks]), (j / C::KS) & 1, abort_flag, to, ROLE_MMA)) break;
+          if (j >= 2 && !wait_bounded(smem_u32(&bars->s_free[sb]), ((j - 2) >> 1) & 1, abort_flag, to, ROLE_MMA))
+            break;
+          tc_fence_after();
+          const uint32_t d_s = tmem + (sb ? SKV_TM_S1 : SKV_TM_S0);
+          const uint32_t kbase = sK + ks * C::TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+            mma_ss(d_s, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024), IDESC_S,
+                   kk > 0 ? 1u : 0u);
+          }
+          mma_commit(smem_u32(&bars->s_full[sb]));
+          mma_commit(smem_u32(&bars->k_empty[ks]));
+        }
+        if (j >= 1) {
+          const int i = j - 1;
+          const int vs = i % C::VS;
+          if (!wait_bounded(b_p, i & 1, abort_flag, to, ROLE_MMA)) break;
+          if (!wait_bounded(smem_u32(&bars->v_full[vs]), (i / C::VS) & 1, abort_flag, to, ROLE_MMA)) break;
+          tc_fence_after();
+          const uint32_t vbase = sV + vs * C::TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_ts(tmem + SKV_TM_O, tmem + SKV_TM_P + kk * 8,
+                   smem_desc_sw128(vbase + kk * 2048, C::CHUNK_BYTES, 1024), IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(smem_u32(&bars->v_empty[vs]));
+          mma_commit(b_pv);
+        }
+      }
+      mma_commit(b_final);
+      wait_drain(b_final, 0, to);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps 0..3
+    const int r = threadIdx.x;
+    const int row = q_first + r;
+    const int pos = offset + row;  // sequence position of this query row
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float c_log2 = p.scale_log2;
+    const uint64_t cc = f2_pack(c_log2, c_log2);
+    // A warp whose 32 rows are all past Nq has nothing to store: it only
+    // keeps the hand-offs going.
+    const bool live = q_first + warp * 32 < p.Nq;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int i = 0; i < nkv; ++i) {
+      const int sb = i & 1;
+      ok = wait_warp(smem_u32(&bars->s_full[sb]), (i >> 1) & 1, abort_flag, to);
+      if (!ok) break;
+      tc_fence_after();
+      const int kv0 = (kt_begin + i) * BN;
+      uint32_t pk[2][32];
+      float alpha = 1.f, rowsum = 0.f, m_new = m;
+      bool rescale = false;
+      if (live) {
+        uint32_t s[128];
+        const uint32_t s_addr = lane_addr + (sb ? SKV_TM_S1 : SKV_TM_S0);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[sb]));
+        // Mask: keys past the row's position (causal) or past Nk.
+        const int lim = CAUSAL ? min(pos, p.Nk - 1) - kv0 : p.Nk - 1 - kv0;
+        if (lim < BN - 1) {
+#pragma unroll
+          for (int e = 0; e < 128; ++e)
+            if (e > lim) s[e] = __float_as_uint(-INFINITY);
+        }
+        float mx8[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx8[a] = __uint_as_float(s[a]);
+#pragma unroll
+        for (int e = 8; e < 128; e += 16)
+#pragma unroll
+          for (int a = 0; a < 8; ++a)
+            mx8[a] = fmax3(mx8[a], __uint_as_float(s[e + a]), __uint_as_float(s[e + 8 + a]));
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+        const float m_cand = mx * c_log2;
+        if (m_cand > m + RESCALE_THRESHOLD) m_new = m_cand;
+        rescale = (i > 0) && (m_new != m);
+        alpha = rescale ? ex2(m - m_new) : 1.f;
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        const uint64_t mm = f2_pack(-m_use, -m_use);
+        uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const uint64_t x =
+                f2_fma(f2_pack(__uint_as_float(s[c * 32 + e]), __uint_as_float(s[c * 32 + e + 1])), cc, mm);
+            float x0, x1;
+            f2_unpack(x, x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            acc[(e >> 1) & 3] = f2_add(acc[(e >> 1) & 3], f2_pack(p0, p1));
+            pk[c >> 1][(c & 1) * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
+          }
+        }
+        float r0, r1, r2, r3;
+        f2_unpack(f2_add(acc[0], acc[1]), r0, r1);
+        f2_unpack(f2_add(acc[2], acc[3]), r2, r3);
+        rowsum = (r0 + r1) + (r2 + r3);
+      } else {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[sb]));
+      }
+      if (i > 0) {
+        // O and the P buffer are in use by PV(i-1) until it completes.
+        ok = wait_warp(b_pv, (i - 1) & 1, abort_flag, to);
+        if (!ok) break;
+        tc_fence_after();
+        if (live && __any_sync(0xffffffffu, rescale)) {
+          const uint64_t aa = f2_pack(alpha, alpha);
+#pragma unroll
+          for (int c = 0; c < HD / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + SKV_TM_O + c * 32, o);
+            tmem_wait_ld();
+            reg_fence32(o);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float a0, a1;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), aa), a0, a1);
+              o[e] = __float_as_uint(a0);
+              o[e + 1] = __float_as_uint(a1);
+            }
+            tmem_st32(lane_addr + SKV_TM_O + c * 32, o);
+          }
+        }
+      }
+      if (live) {
+        tmem_st32(lane_addr + SKV_TM_P, pk[0]);
+        tmem_st32(lane_addr + SKV_TM_P + 32, pk[1]);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_p);
+      l = l * alpha + rowsum;
+      m = m_new;
+    }
+    if (ok) ok = wait_warp(b_pv, (nkv - 1) & 1, abort_flag, to);
+    if (ok && live) {
+      tc_fence_after();
+      uint32_t o[HD / 32][32];
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) tmem_ld32(lane_addr + SKV_TM_O + c * 32, o[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) reg_fence32(o[c]);
+      if (row < p.Nq) {
+        const size_t prow = (static_cast<size_t>(split) * p.BH + bh) * p.Nq + row;
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        const float lse_row = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (p.direct) {
+          // One range: this is the final result (prow = bh * Nq + row).
+          uint4* dst = reinterpret_cast<uint4*>(p.o + prow * HD);
+#pragma unroll
+          for (int c = 0; c < HD / 32; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; e += 8)
+              dst[c * 4 + e / 8] = make_uint4(
+                  pack_bf16x2(__uint_as_float(o[c][e]) * inv_l, __uint_as_float(o[c][e + 1]) * inv_l),
+                  pack_bf16x2(__uint_as_float(o[c][e + 2]) * inv_l, __uint_as_float(o[c][e + 3]) * inv_l),
+                  pack_bf16x2(__uint_as_float(o[c][e + 4]) * inv_l, __uint_as_float(o[c][e + 5]) * inv_l),
+                  pack_bf16x2(__uint_as_float(o[c][e + 6]) * inv_l, __uint_as_float(o[c][e + 7]) * inv_l));
+          p.lse[prow] = lse_row;
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.o_part + prow * HD);
+#pragma unroll
+          for (int c = 0; c < HD / 32; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              dst[c * 8 + e / 4] =
+                  make_float4(__uint_as_float(o[c][e]) * inv_l, __uint_as_float(o[c][e + 1]) * inv_l,
+                              __uint_as_float(o[c][e + 2]) * inv_l, __uint_as_float(o[c][e + 3]) * inv_l);
+          p.lse_part[prow] = lse_row;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == SKV_MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Merge of the partial results: one warp per query row; lane l holds
+// columns [l*HD/32, (l+1)*HD/32).
+template <int HD>
+__global__ void __launch_bounds__(128) fa2_splitkv_combine_kernel(const float* __restrict__ o_part,
+                                                                  const float* __restrict__ lse_part,
+                                                                  __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
+                                                                  int rows, int n_splits) {
+  const int row = static_cast<int>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  constexpr int PER = HD / 32;  // 4 (d = 128) or 2 (d = 64) columns per lane
+  float mx = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) mx = fmaxf(mx, lse_part[static_cast<size_t>(s) * rows + row]);
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  float wsum = 0.f;
+  if (mx != -INFINITY) {
+    for (int s = 0; s < n_splits; ++s) {
+      const float ls = lse_part[static_cast<size_t>(s) * rows + row];
+      if (ls == -INFINITY) continue;  // a range with no visible key
+      const float w = __expf(ls - mx);
+      wsum += w;
+      const float* src = o_part + (static_cast<size_t>(s) * rows + row) * HD + lane * PER;
+      if constexpr (PER == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(src);
+        acc[0] += w * x.x;
+        acc[1] += w * x.y;
+        acc[2] += w * x.z;
+        acc[3] += w * x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2*>(src);
+        acc[0] += w * x.x;
+        acc[1] += w * x.y;
+      }
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  __nv_bfloat16* dst = o + static_cast<size_t>(row) * HD + lane * PER;
+  if constexpr (PER == 4) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv),
+                                                pack_bf16x2(acc[2] * inv, acc[3] * inv));
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  }
+  if (lane == 0) lse[row] = (wsum > 0.f) ? mx + logf(wsum) : -INFINITY;
+}

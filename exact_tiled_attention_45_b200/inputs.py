@@ -10,7 +10,7 @@ from __future__ import annotations
 
 import torch
 
-__all__ = ["make_qkv", "Workload", "WORKLOADS"]
+__all__ = ["make_qkv", "make_q_kv", "Workload", "DecodeWorkload", "WORKLOADS"]
 
 
 def make_qkv(B: int, H: int, N: int, d: int, seed: int = 0, qk_mult: float = 1.0):
@@ -20,6 +20,22 @@ def make_qkv(B: int, H: int, N: int, d: int, seed: int = 0, qk_mult: float = 1.0
     q = torch.randn(B, H, N, d, generator=g, dtype=torch.float32).to(torch.bfloat16)
     k = torch.randn(B, H, N, d, generator=g, dtype=torch.float32).to(torch.bfloat16)
     v = torch.randn(B, H, N, d, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    if qk_mult != 1.0:
+        q = q * qk_mult
+        k = k * qk_mult
+    return q, k, v
+
+
+def make_q_kv(B: int, H: int, Nq: int, Nk: int, d: int, seed: int = 0, qk_mult: float = 1.0):
+    """Q [B, H, Nq, d] and K, V [B, H, Nk, d] (bf16, CPU), drawn in that order.
+
+    Same recipe as :func:`make_qkv`, which it equals when Nq == Nk.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    q = torch.randn(B, H, Nq, d, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    k = torch.randn(B, H, Nk, d, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    v = torch.randn(B, H, Nk, d, generator=g, dtype=torch.float32).to(torch.bfloat16)
     if qk_mult != 1.0:
         q = q * qk_mult
         k = k * qk_mult
@@ -48,6 +64,40 @@ class Workload:
         return f"Workload({self.as_dict()})"
 
 
+class DecodeWorkload:
+    """Nq queries (the last Nq positions) against Nk keys per (batch, head)."""
+
+    def __init__(self, name: str, B: int, H: int, Nq: int, Nk: int, d: int, causal: bool, qk_mult: float = 1.0):
+        self.name, self.B, self.H, self.Nq, self.Nk, self.d = name, B, H, Nq, Nk, d
+        self.causal, self.qk_mult = bool(causal), float(qk_mult)
+
+    @property
+    def pairs(self) -> int:
+        """Allowed (query, key) pairs per head."""
+        if not self.causal:
+            return self.Nq * self.Nk
+        off = self.Nk - self.Nq
+        return sum(off + i + 1 for i in range(self.Nq))
+
+    @property
+    def flops(self) -> float:
+        """4 * d FLOP per allowed (query, key) pair (two dot products of length d)."""
+        return 4.0 * self.B * self.H * self.pairs * self.d
+
+    @property
+    def bytes(self) -> float:
+        """Algorithmic HBM bytes: read Q, K, V once (bf16), write O (bf16) and LSE (fp32)."""
+        bh = self.B * self.H
+        return bh * (2 * self.Nq * self.d * 2 + 2 * self.Nk * self.d * 2 + self.Nq * 4)
+
+    def as_dict(self) -> dict:
+        return {"workload": self.name, "B": self.B, "H": self.H, "Nq": self.Nq, "Nk": self.Nk,
+                "d": self.d, "causal": self.causal, "qk_mult": self.qk_mult}
+
+    def __repr__(self) -> str:  # pragma: no cover
+        return f"DecodeWorkload({self.as_dict()})"
+
+
 def _grid():
     out = []
     for d in (64, 128):
@@ -71,3 +121,10 @@ for _N in (512, 1024, 2048, 4096, 8192, 16384):
     WORKLOADS[_w.name] = _w
 for _w in _grid():
     WORKLOADS.setdefault(_w.name, _w)
+
+#: Few queries against a long key sequence (split-K/V entry point).
+for _w in (DecodeWorkload("decode_B8_H16_Nk16384_d128", 8, 16, 1, 16384, 128, True),
+           DecodeWorkload("decode_B1_H16_Nk65536_d128", 1, 16, 1, 65536, 128, True),
+           DecodeWorkload("decode_B32_H16_Nk4096_d64", 32, 16, 1, 4096, 64, True),
+           DecodeWorkload("chunk_B1_H16_Nq512_Nk16384_d128", 1, 16, 512, 16384, 128, True)):
+    WORKLOADS[_w.name] = _w

@@ -59,7 +59,8 @@ typedef enum {
  *             is masked).
  *   d       : head dimension, 64 or 128 (others -> FA2_ERR_UNSUPPORTED).
  *   causal  : 0 = every key; non-zero = key j allowed only for query i >= j.
- *   scale   : multiplier of q.k (finite; the usual choice is 1/sqrt(d)).
+ *   scale   : multiplier of q.k, finite and > 0 (the usual choice is
+ *             1/sqrt(d)); other values -> FA2_ERR_INVALID_ARG.
  *   stream  : cudaStream_t as void* (NULL = legacy default stream).
  */
 int fa2_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
@@ -96,6 +97,60 @@ int fa2_sync_status(void* stream);
  */
 int fa2_fwd_inject_timeout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                            int N, int d, int causal, float scale, unsigned long long timeout_ns, void* stream);
+
+/*
+ * Exact attention of few queries against many keys: decoding, or a chunk of
+ * new queries after a cached prefix.  The pages separate the processing of a
+ * long prompt from token-by-token generation, whose bottlenecks differ
+ * (iplexlaw blog "FlashAttention-2: making long-context attention run
+ * efficiently on GPUs", section "Document the implementation difference").
+ * With few query rows, one CTA per query tile and head would leave most SMs
+ * idle, so the keys are split into ranges: one CTA per (128-row query tile,
+ * batch*head, key range) computes that range's partial output and
+ * logsumexp, and a second kernel merges them exactly
+ * (LSE = ln sum_r exp(LSE_r), O = sum_r exp(LSE_r - LSE) O_r).
+ *
+ *   q       : device pointer, bf16 [B,H,Nq,d], contiguous, 16-byte aligned.
+ *   k, v    : device pointers, bf16 [B,H,Nk,d], contiguous, 16-byte aligned.
+ *   o       : device pointer, bf16 [B,H,Nq,d]; written.
+ *   lse     : device pointer, fp32 [B,H,Nq], 4-byte aligned; written (natural
+ *             log of the sum of exp of the scaled scores over allowed keys).
+ *   Nq, Nk  : 1 <= Nq <= Nk.  Query row i is sequence position Nk - Nq + i
+ *             (the last Nq positions); with Nq == Nk this is fa2_fwd.
+ *   B, H    : >= 1 with B*H <= 65535.
+ *   d       : 64 or 128 (others -> FA2_ERR_UNSUPPORTED).
+ *   causal  : 0 = every key; non-zero = key j allowed for query row i only if
+ *             j <= Nk - Nq + i.
+ *   scale   : finite and > 0.
+ *   n_splits: number of key ranges; 0 lets the library choose: the fewest
+ *             ranges that give at least 0.8 x (SM count) CTAs, keeping at
+ *             least 4 key tiles per range.  A request is capped at 128 and at
+ *             the number of 128-key tiles; fa2_fwd_splitkv_splits returns the
+ *             count used.
+ *   workspace, workspace_bytes: caller-owned device buffer, 256-byte aligned,
+ *             of at least fa2_fwd_splitkv_workspace_bytes(...) bytes (same
+ *             sizes and n_splits), holding the fp32 partial outputs and
+ *             logsumexps between the two kernels.  It must not overlap any
+ *             other argument.  Concurrent calls need separate workspaces.
+ *             With a single range the kernel writes o and lse itself, no
+ *             merge runs, the required size is 0 and workspace may be NULL.
+ *   stream  : cudaStream_t as void*; the kernels are queued on it.
+ * Argument errors are reported before anything is launched; kernel-side
+ * timeouts through fa2_sync_status.  The library allocates nothing.
+ */
+int fa2_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                    int d, int causal, float scale, int n_splits, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/* Key ranges fa2_fwd_splitkv uses for these sizes and request (0 on bad sizes). */
+int fa2_fwd_splitkv_splits(int B, int H, int Nq, int Nk, int d, int n_splits);
+
+/*
+ * Workspace bytes fa2_fwd_splitkv needs for these sizes and request: 0 when a
+ * single range is used (no workspace needed) and 0 on bad sizes, which
+ * fa2_fwd_splitkv_splits tells apart (it returns 0 only on bad sizes).
+ */
+size_t fa2_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int n_splits);
 
 /* Static description of a status code. */
 const char* fa2_strerror(int status);

@@ -108,3 +108,84 @@ def test_python_wrapper_rejects_wrong_tensors():
         binding._check_qkv(q.transpose(2, 3), q, q, "cpu")
     with pytest.raises(ValueError):
         binding._check_qkv(q, q, q, "cuda")
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.125])
+def test_non_positive_scale_rejected(lib, scale):
+    # Masked scores are -inf before scaling; a scale <= 0 would turn them into
+    # NaN or +inf, so the library refuses it.
+    assert _call(lib, scale=scale) == binding.FA2_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------- split-K/V
+
+def _skv(lib, q=FAKE, k=FAKE + (1 << 32), v=FAKE + (2 << 32), o=FAKE + (3 << 32), lse=FAKE + (4 << 32),
+         B=1, H=2, Nq=1, Nk=1000, d=128, causal=0, scale=0.125, n_splits=0, ws=FAKE + (5 << 32), ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = 1 << 30
+    return lib.fa2_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, n_splits, ws, ws_bytes, None)
+
+
+def test_splitkv_split_count_and_workspace(lib):
+    n_kv = 8  # Nk = 1000 -> 8 key tiles of 128
+    for req, want in ((1, 1), (2, 2), (3, 3), (5, 4), (7, 4), (8, 8), (9, 8), (500, 8)):
+        # a request of s ranges means ceil(8/s) tiles per range, which may
+        # cover the 8 tiles with fewer ranges (5 -> 2 tiles each -> 4 ranges)
+        got = lib.fa2_fwd_splitkv_splits(1, 2, 1, 1000, 128, req)
+        assert got == want, (req, got)
+    assert lib.fa2_fwd_splitkv_splits(1, 2, 1, 1000, 128, 1) == 1
+    auto = lib.fa2_fwd_splitkv_splits(1, 2, 1, 1000, 128, 0)
+    assert 1 <= auto <= n_kv
+    # workspace: fp32 partial O then fp32 partial LSE, each rounded to 256 bytes
+    s = lib.fa2_fwd_splitkv_splits(2, 3, 5, 1000, 64, 3)
+    assert s == 3
+    rows = s * 2 * 3 * 5
+    r256 = lambda x: (x + 255) // 256 * 256
+    assert lib.fa2_fwd_splitkv_workspace_bytes(2, 3, 5, 1000, 64, 3) == r256(rows * 64 * 4) + r256(rows * 4)
+    for bad in ((1, 1, 0, 10, 64, 0), (1, 1, 11, 10, 64, 0), (1, 1, 1, 10, 96, 0), (1, 1, 1, 10, 64, -1),
+                (300, 300, 1, 10, 64, 0)):
+        assert lib.fa2_fwd_splitkv_workspace_bytes(*bad) == 0
+        assert lib.fa2_fwd_splitkv_splits(*bad) == 0
+
+
+def test_splitkv_auto_split_choice(lib):
+    # The choice assumes a B200 (148 SMs) when no device can be queried, and a
+    # B200 is what the library targets: the fewest ranges giving >= 119 CTAs,
+    # with at least 4 key tiles per range.
+    assert lib.fa2_fwd_splitkv_splits(8, 16, 1, 16384, 128, 0) == 1      # 128 heads fill the GPU
+    assert lib.fa2_fwd_splitkv_splits(1, 16, 1, 65536, 128, 0) == 8      # 16 heads x 8 ranges
+    assert lib.fa2_fwd_splitkv_splits(1, 1, 1, 65536, 128, 0) == 103    # ceil(512 / ceil(512 / 119))
+    assert lib.fa2_fwd_splitkv_splits(1, 1, 1, 1000, 128, 0) == 2        # only 8 tiles: >= 4 per range
+    assert lib.fa2_fwd_splitkv_splits(1, 16, 512, 16384, 128, 0) == 2    # 4 query tiles x 16 heads
+    # one range: no workspace, the kernel writes O and LSE itself
+    assert lib.fa2_fwd_splitkv_workspace_bytes(8, 16, 1, 16384, 128, 0) == 0
+    assert lib.fa2_fwd_splitkv_workspace_bytes(8, 16, 1, 16384, 128, 1) == 0
+    assert lib.fa2_fwd_splitkv_workspace_bytes(8, 16, 1, 16384, 128, 2) > 0
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=0), binding.FA2_ERR_INVALID_ARG),
+    (dict(ws=0, n_splits=2), binding.FA2_ERR_INVALID_ARG),          # two ranges need a workspace
+    (dict(Nq=0), binding.FA2_ERR_INVALID_ARG),
+    (dict(Nq=1001), binding.FA2_ERR_INVALID_ARG),          # Nq > Nk
+    (dict(B=300, H=300), binding.FA2_ERR_INVALID_ARG),     # B*H > 65535
+    (dict(n_splits=-1), binding.FA2_ERR_INVALID_ARG),
+    (dict(scale=0.0), binding.FA2_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), binding.FA2_ERR_INVALID_ARG),
+    (dict(d=96), binding.FA2_ERR_UNSUPPORTED),
+    (dict(ws=FAKE + (5 << 32) + 128), binding.FA2_ERR_INVALID_ARG),  # workspace not 256-aligned
+    (dict(ws_bytes=1024), binding.FA2_ERR_INVALID_ARG),              # workspace too small
+    (dict(o=FAKE + (1 << 32)), binding.FA2_ERR_INVALID_ARG),         # o aliases k
+    (dict(ws=FAKE + (2 << 32)), binding.FA2_ERR_INVALID_ARG),        # workspace aliases v
+])
+def test_splitkv_bad_arguments_rejected_before_launch(lib, kw, expect):
+    assert _skv(lib, **kw) == expect
+    assert lib.fa2_last_error_detail()
+
+
+def test_splitkv_wrapper_shape_checks():
+    import torch
+    q = torch.zeros(1, 2, 4, 64, dtype=torch.bfloat16)
+    kv = torch.zeros(1, 2, 9, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):  # tensors on the CPU
+        binding._check_q_kv(q, kv, kv)
