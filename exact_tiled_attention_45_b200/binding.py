@@ -22,7 +22,8 @@ FA2_OK, FA2_ERR_INVALID_ARG, FA2_ERR_UNSUPPORTED, FA2_ERR_CUDA, FA2_ERR_TIMEOUT 
 #: Every symbol the header declares.
 EXPORTS = ("fa2_fwd", "fa2_fwd_host", "fa2_fwd_host_workspace_bytes", "fa2_sync_status",
            "fa2_fwd_inject_timeout", "fa2_fwd_splitkv", "fa2_fwd_splitkv_splits",
-           "fa2_fwd_splitkv_workspace_bytes", "fa2_strerror", "fa2_last_error_detail", "fa2_version")
+           "fa2_fwd_splitkv_workspace_bytes", "fa2_fwd_splitkv_static", "fa2_strerror", "fa2_last_error_detail",
+           "fa2_version")
 
 _lib = None
 
@@ -55,6 +56,9 @@ def load() -> ctypes.CDLL:
     lib.fa2_fwd_splitkv_splits.restype = _int
     lib.fa2_fwd_splitkv_workspace_bytes.argtypes = [_int] * 6
     lib.fa2_fwd_splitkv_workspace_bytes.restype = ctypes.c_size_t
+    lib.fa2_fwd_splitkv_static.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _float,
+                                           _int, _vp]
+    lib.fa2_fwd_splitkv_static.restype = _int
     lib.fa2_strerror.argtypes = [_int]
     lib.fa2_strerror.restype = ctypes.c_char_p
     lib.fa2_last_error_detail.argtypes = []
@@ -233,5 +237,37 @@ def fwd_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool 
     st = lib.fa2_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                              B, H, Nq, Nk, d, int(bool(causal)), float(scale), int(n_splits),
                              ws_ptr, ws_len, _stream_handle(stream))
+    _check(st, lib)
+    return out, lse
+
+
+#: Bytes of the library's own scratch array used by :func:`fwd_splitkv_static`.
+SPLITKV_STATIC_SCRATCH_BYTES = 16 << 20
+
+
+def fwd_splitkv_static(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+                       scale: float | None = None, n_splits: int = 0, out: torch.Tensor | None = None,
+                       lse: torch.Tensor | None = None, stream=None):
+    """:func:`fwd_splitkv` with the partials in the library's fixed 16 MiB
+    scratch array instead of a caller workspace.
+
+    For callers that may not allocate device memory themselves.  The C entry
+    point allocates nothing; this wrapper only allocates ``out`` and ``lse``
+    when they are not given.  Calls that overlap on the GPU race on the shared
+    scratch; the first call on a device should precede any stream capture.
+    """
+    lib = load()
+    _check_q_kv(q, k, v)
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    st = lib.fa2_fwd_splitkv_static(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                    B, H, Nq, Nk, d, int(bool(causal)), float(scale), int(n_splits),
+                                    _stream_handle(stream))
     _check(st, lib)
     return out, lse

@@ -46,6 +46,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "fa2.h"
 #include "sm100_ptx.cuh"
@@ -913,6 +914,47 @@ static int splitkv_impl(const void* q, const void* k, const void* v, void* o, fl
                 : skv_launch_t<128, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
 }
 
+// ------------------------------------------------------------------ split-K/V with library-owned scratch
+// For callers that cannot allocate device memory (see fa2_fwd_splitkv_static
+// in fa2.h): the partial outputs live in this fixed array instead of a
+// caller workspace.  Every device that loads the library holds it until the
+// process exits.  Nothing in it has to start at zero: each call writes every
+// partial the merge reads.  All calls share it, so calls that overlap on the
+// GPU (other streams, other host threads) race on its contents.
+static __device__ __align__(256) unsigned char g_skv_static_scratch[FA2_SPLITKV_STATIC_SCRATCH_BYTES];
+
+constexpr int MAX_DEVICES = 64;
+static std::mutex g_static_scratch_mu;
+static void* g_static_scratch_addr[MAX_DEVICES] = {};
+
+// Device address of the scratch array on the current device.  The host-side
+// name g_skv_static_scratch is only a stand-in for the symbol; the address is
+// looked up once per device (the first call on that device) and cached.
+static int static_scratch_on_current_device(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    set_detail("cudaGetDevice: %s", cudaGetErrorString(e));
+    return FA2_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= MAX_DEVICES) {
+    set_detail("device %d is beyond the %d devices the static scratch table covers", dev, MAX_DEVICES);
+    return FA2_ERR_UNSUPPORTED;
+  }
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (!g_static_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_skv_static_scratch);
+    if (e != cudaSuccess || !ptr) {
+      set_detail("cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
+      return FA2_ERR_CUDA;
+    }
+    g_static_scratch_addr[dev] = ptr;
+  }
+  *out = g_static_scratch_addr[dev];
+  return FA2_OK;
+}
+
 }  // namespace fa2
 
 // ====================================================================== C ABI
@@ -1018,6 +1060,34 @@ int fa2_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float*
                     int d, int causal, float scale, int n_splits, void* workspace, size_t workspace_bytes,
                     void* stream) {
   return fa2::splitkv_impl(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, n_splits, workspace, workspace_bytes,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int fa2_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                           int Nk, int d, int causal, float scale, int n_splits, void* stream) {
+  fa2::g_detail[0] = 0;
+  if (!q || !k || !v || !o || !lse) {
+    fa2::set_detail("null pointer");
+    return FA2_ERR_INVALID_ARG;
+  }
+  size_t need = 0;
+  if (fa2::skv_sizes_ok(B, H, Nq, Nk) && n_splits >= 0 && (d == 64 || d == 128)) {
+    const int splits = fa2::skv_resolve_splits(B, H, Nq, Nk, n_splits);
+    need = fa2::skv_workspace_bytes(B, H, Nq, d, splits);
+    if (need > FA2_SPLITKV_STATIC_SCRATCH_BYTES) {
+      fa2::set_detail("%d key ranges need %zu bytes of scratch; the static scratch holds %zu (fewer ranges need "
+                      "less, one range none; fa2_fwd_splitkv takes a caller workspace of any size)",
+                      splits, need, static_cast<size_t>(FA2_SPLITKV_STATIC_SCRATCH_BYTES));
+      return FA2_ERR_INVALID_ARG;
+    }
+  }
+  void* scratch = nullptr;
+  if (need > 0) {
+    const int st = fa2::static_scratch_on_current_device(&scratch);
+    if (st != FA2_OK) return st;
+  }
+  return fa2::splitkv_impl(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, n_splits, scratch,
+                           scratch ? static_cast<size_t>(FA2_SPLITKV_STATIC_SCRATCH_BYTES) : 0,
                            static_cast<cudaStream_t>(stream));
 }
 

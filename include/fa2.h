@@ -152,6 +152,38 @@ int fa2_fwd_splitkv_splits(int B, int H, int Nq, int Nk, int d, int n_splits);
  */
 size_t fa2_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int n_splits);
 
+/*
+ * fa2_fwd_splitkv without a workspace argument, for callers that cannot
+ * allocate device memory: a plug-in running inside a host application whose
+ * memory pool owns the whole device (a serving process or a framework's
+ * caching allocator), where a direct cudaMalloc would bypass that pool or be
+ * refused, and latency-critical loops where an allocation could stall the
+ * device.  The pages have no counterpart: this is a property of the library,
+ * not of the method.
+ *
+ * Arguments, layout and results are those of fa2_fwd_splitkv.  The partial
+ * outputs go to a scratch array inside the library (a file-scope device
+ * array of FA2_SPLITKV_STATIC_SCRATCH_BYTES = 16 MiB that every GPU which
+ * loads the library holds until the process exits).  The library allocates
+ * nothing on this path: no cudaMalloc, no cudaFree, no allocating library
+ * call.
+ *
+ *   - A request whose partials need more than 16 MiB (see
+ *     fa2_fwd_splitkv_workspace_bytes) returns FA2_ERR_INVALID_ARG before
+ *     anything is launched; fewer key ranges need less, and one range needs
+ *     none.
+ *   - The first call on each device that needs the scratch looks up the
+ *     array's device address there (cudaGetSymbolAddress) and caches it;
+ *     make that first call before any stream capture.
+ *   - Every call shares the one array, which keeps the last call's contents.
+ *     Nothing in it has to start at zero (each call writes every partial
+ *     before its merge reads it), but calls that overlap on the GPU (on other
+ *     streams or from other host threads) race on it: serialise them.
+ */
+#define FA2_SPLITKV_STATIC_SCRATCH_BYTES (16u << 20)
+int fa2_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                           int Nk, int d, int causal, float scale, int n_splits, void* stream);
+
 /* Static description of a status code. */
 const char* fa2_strerror(int status);
 

@@ -189,3 +189,13 @@ def test_splitkv_wrapper_shape_checks():
     kv = torch.zeros(1, 2, 9, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):  # tensors on the CPU
         binding._check_q_kv(q, kv, kv)
+
+
+def test_static_scratch_entry_rejects_on_the_host(lib):
+    # beyond the 16 MiB scratch: 32 ranges x 16 heads x 4096 rows x (128 + 1) floats
+    rc = lib.fa2_fwd_splitkv_static(FAKE, FAKE + (1 << 32), FAKE + (2 << 32), FAKE + (3 << 32), FAKE + (4 << 32),
+                                    1, 16, 4096, 4096, 128, 1, 0.088, 32, None)
+    assert rc == binding.FA2_ERR_INVALID_ARG
+    assert b"static scratch" in lib.fa2_last_error_detail()
+    rc = lib.fa2_fwd_splitkv_static(0, FAKE, FAKE, FAKE, FAKE, 1, 1, 1, 128, 64, 0, 0.125, 0, None)
+    assert rc == binding.FA2_ERR_INVALID_ARG
