@@ -18,7 +18,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libfa2.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 SOURCES = [os.path.join(CSRC, "fa2_fwd.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, "sm100_ptx.cuh"), os.path.join(INCLUDE, "fa2.h")]
+DEPS = SOURCES + [os.path.join(CSRC, "sm100_ptx.cuh"), os.path.join(CSRC, "fa2_splitkv.cuh"),
+                  os.path.join(INCLUDE, "fa2.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

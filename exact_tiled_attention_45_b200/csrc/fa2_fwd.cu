@@ -11,7 +11,8 @@
 //          with the softmax scale folded into one FMA, and only the diagonal
 //          (causal) or ragged tail tile is masked element by element;
 //      (2) parallel over the sequence: one CTA per (256-row query block, head,
-//          batch);
+//          batch); with causal masking the blocks of a group of heads launch
+//          heaviest first;
 //      (3) work split without shared-memory reductions: each softmax thread
 //          owns one query row (one TMEM lane) from scores to output.
 //  * iplexlaw blog, section "Tiling preserves the attention calculation":
@@ -129,9 +130,10 @@ struct Params {
   __nv_bfloat16* o;
   float* lse;
   int N;
-  int H;
-  int n_q_blocks;  // 256-row query blocks
-  int n_kv_tiles;  // 128-key tiles
+  int BH;           // B * H
+  int n_q_blocks;   // 256-row query blocks
+  int n_kv_tiles;   // 128-key tiles
+  int group_heads;  // heads per launch-order group (see the kernel's work mapping)
   float scale_log2;  // scale * log2(e)
   unsigned long long timeout_ns;
   int inject_timeout;  // test hook: withhold the Q loads
@@ -387,8 +389,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int qb = CAUSAL ? (p.n_q_blocks - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
-  const int bh = static_cast<int>(blockIdx.z) * p.H + static_cast<int>(blockIdx.y);
+  // Work mapping of the 1-D grid (CTAs launch roughly in index order): the
+  // heads are taken in groups of group_heads; within a group the query-block
+  // rank is the slow index and the head the fast one.  With causal masking
+  // rank 0 is the heaviest block, so each group runs longest-first and the
+  // last wave holds the lightest blocks; a group's K/V stays small enough to
+  // be reused from L2 by its blocks.  Without masking every block costs the
+  // same and group_heads = 1 (all blocks of a head in a row).
+  const int per_group = p.group_heads * p.n_q_blocks;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int in_grp = static_cast<int>(blockIdx.x) - grp * per_group;
+  const int grp_heads = min(p.group_heads, p.BH - grp * p.group_heads);
+  const int rank = in_grp / grp_heads;
+  const int bh = grp * p.group_heads + (in_grp - rank * grp_heads);
+  const int qb = CAUSAL ? (p.n_q_blocks - 1 - rank) : rank;
   const int q0 = qb * BLOCK_M;
   const int n0 = kv_tiles_for<CAUSAL>(qb, 0, p.n_kv_tiles);
   const int n1 = kv_tiles_for<CAUSAL>(qb, 1, p.n_kv_tiles);  // n0 <= n1
@@ -668,8 +682,9 @@ static int validate(const void* q, const void* k, const void* v, const void* o, 
     set_detail("null pointer");
     return FA2_ERR_INVALID_ARG;
   }
-  if (B < 1 || H < 1 || N < 1 || B > 65535 || H > 65535) {
-    set_detail("bad sizes B=%d H=%d N=%d", B, H, N);
+  if (B < 1 || H < 1 || N < 1 || B > 65535 || H > 65535 ||
+      static_cast<long long>(B) * H * ((N + BLOCK_M - 1) / BLOCK_M) > 0x7fffffffLL) {
+    set_detail("bad sizes B=%d H=%d N=%d (need B, H <= 65535 and B*H*ceil(N/256) < 2^31)", B, H, N);
     return FA2_ERR_INVALID_ARG;
   }
   if (!std::isfinite(scale) || !(scale > 0.f)) {
@@ -716,7 +731,7 @@ static int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
     }
     if (dev < 32) attr_done_mask |= (1 << dev);
   }
-  dim3 grid(prm.n_q_blocks, H, B);
+  dim3 grid(B * H * prm.n_q_blocks);
   kern<<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -724,6 +739,29 @@ static int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
     return FA2_ERR_CUDA;
   }
   return FA2_OK;
+}
+
+static int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) ==
+                                                 cudaSuccess && n > 0)
+    return n;
+  cudaGetLastError();  // no device here: plan for a B200
+  return 148;
+}
+
+// Heads per launch-order group for causal masking: enough heads that the
+// last group spans two waves of CTAs (so it can run longest-first), few
+// enough that the group's K and V (4*N*d bytes per head) stay within 48 MiB
+// of L2, then evened out over the groups.
+static int causal_group_heads(int BH, int N, int d, int n_q_blocks) {
+  const int sms = sm_count();
+  int g = (2 * sms + n_q_blocks - 1) / n_q_blocks;
+  const long long kv_head = 4LL * N * d;
+  const long long g_l2 = std::max(1LL, (48LL << 20) / kv_head);
+  g = static_cast<int>(std::min<long long>(std::min<long long>(g, g_l2), BH));
+  const int groups = (BH + g - 1) / g;
+  return (BH + groups - 1) / groups;
 }
 
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
@@ -741,9 +779,10 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
   prm.N = N;
-  prm.H = H;
+  prm.BH = BH;
   prm.n_q_blocks = (N + BLOCK_M - 1) / BLOCK_M;
   prm.n_kv_tiles = (N + BN - 1) / BN;
+  prm.group_heads = causal ? causal_group_heads(BH, N, d, prm.n_q_blocks) : 1;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
   prm.timeout_ns = timeout_ns;
   prm.inject_timeout = inject;
@@ -759,15 +798,6 @@ constexpr unsigned long long DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s per wai
 // ------------------------------------------------------------------ split-K/V host side
 
 constexpr int SKV_MAX_SPLITS = 128;
-
-static int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) ==
-                                                 cudaSuccess && n > 0)
-    return n;
-  cudaGetLastError();  // no device here: plan for a B200
-  return 148;
-}
 
 static bool skv_sizes_ok(int B, int H, int Nq, int Nk) {
   return B >= 1 && H >= 1 && Nq >= 1 && Nk >= Nq && static_cast<long long>(B) * H <= 65535;

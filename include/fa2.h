@@ -55,8 +55,8 @@ typedef enum {
  *             written.  Must not overlap q, k, v or lse.
  *   lse     : device pointer, fp32 [B,H,N], contiguous, 4-byte aligned;
  *             written with the natural-log logsumexp of the scaled scores.
- *   B, H, N : >= 1; B <= 65535, H <= 65535.  Any N >= 1 (a ragged last tile
- *             is masked).
+ *   B, H, N : >= 1; B <= 65535, H <= 65535, B*H < 2^31, N <= 16776960.
+ *             Any such N works (a ragged last tile is masked).
  *   d       : head dimension, 64 or 128 (others -> FA2_ERR_UNSUPPORTED).
  *   causal  : 0 = every key; non-zero = key j allowed only for query i >= j.
  *   scale   : multiplier of q.k, finite and > 0 (the usual choice is

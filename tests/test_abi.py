@@ -65,6 +65,8 @@ def _call(lib, q=FAKE, k=FAKE + (1 << 32), v=FAKE + (2 << 32), o=FAKE + (3 << 32
     (dict(B=0), binding.FA2_ERR_INVALID_ARG),
     (dict(H=-1), binding.FA2_ERR_INVALID_ARG),
     (dict(B=70000), binding.FA2_ERR_INVALID_ARG),
+    (dict(B=65535, H=65535), binding.FA2_ERR_INVALID_ARG),   # B*H >= 2^31
+    (dict(B=1024, H=1024, N=2048 * 256), binding.FA2_ERR_INVALID_ARG),  # 2^31 CTAs
     (dict(d=96), binding.FA2_ERR_UNSUPPORTED),
     (dict(d=256), binding.FA2_ERR_UNSUPPORTED),
     (dict(q=FAKE + 8), binding.FA2_ERR_INVALID_ARG),
