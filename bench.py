@@ -55,6 +55,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the timed oracle sample")
     ap.add_argument("--splits", type=int, default=0, help="key ranges for decode workloads (0 = library choice)")
+    ap.add_argument("--no-gemm", action="store_true", help="skip the library GEMM comparator")
     return ap.parse_args()
 
 
@@ -256,6 +257,53 @@ def run_reference(args, w):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def gemm_comparator(w, dev, reps: int = 20) -> dict:
+    """Library bf16 GEMMs on the same GPU, beside the attention kernel.
+
+    The pages put FlashAttention-2 "close to" GEMM efficiency; this measures
+    what the vendor GEMM reaches here: a square 8192^3 matmul, and the two
+    batched GEMMs of unfused attention at the workload's shapes
+    (S = Q K^T, then O = P V, each over all B*H heads, with no softmax and
+    no masking: 4*B*H*N^2*d FLOP).  Timed with CUDA events after warm-up.
+    """
+    import torch
+
+    def timed(fn, flops):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return flops * reps / (e0.elapsed_time(e1) * 1e-3) / 1e12
+
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    a = torch.randn(8192, 8192, device=dev, dtype=torch.bfloat16, generator=g)
+    b = torch.randn(8192, 8192, device=dev, dtype=torch.bfloat16, generator=g)
+    out = {"square_8192_tflops": timed(lambda: a @ b, 2.0 * 8192 ** 3)}
+    del a, b
+    bh = w.B * w.H
+    q = torch.randn(bh, w.N, w.d, device=dev, dtype=torch.bfloat16, generator=g)
+    k = torch.randn(bh, w.N, w.d, device=dev, dtype=torch.bfloat16, generator=g)
+    s = torch.empty(bh, w.N, w.N, device=dev, dtype=torch.bfloat16)
+    o = torch.empty(bh, w.N, w.d, device=dev, dtype=torch.bfloat16)
+
+    def unfused():
+        torch.bmm(q, k.transpose(1, 2), out=s)
+        torch.bmm(s, k, out=o)
+
+    out["bmm_qk_pv_tflops"] = timed(unfused, 4.0 * bh * w.N * w.N * w.d)
+    out["bmm_bytes_of_scores"] = bh * w.N * w.N * 2
+    out["library"] = "torch.matmul / torch.bmm (cuBLAS), bf16 in, bf16 out, fp32 accumulation"
+    del q, k, s, o
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_decode(args, w):
@@ -530,6 +578,10 @@ def main():
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         cpu, _ = cpu_oracle_sample(w, args.cpu_seconds, q_h, k_h, v_h)
+    gemm = None
+    if not args.no_gemm and world == 1:
+        gemm = gemm_comparator(w, dev)
+        gemm["fa2_over_square_gemm"] = achieved / gemm["square_8192_tflops"]
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -547,6 +599,7 @@ def main():
         "gpu_launches": args.steps,
         "e2e": e2e,
         "cpu_baseline": cpu,
+        "gemm_comparator": gemm,
     }
     print(json.dumps(line), flush=True)
     return 0
