@@ -38,6 +38,9 @@ Readings where the pages are silent (each is also listed in the design notes):
 * an empty row (no allowed key; unreachable with N_q == N_k) gives O = 0 and
   LSE = -inf.
 
+The backward (``attention_bwd_ref``) is the chain rule through the same
+three steps, written out at the end of this module.
+
 The oracle is NOT tiled over keys and uses no online softmax: per (b, h) it
 materialises S for a block of query rows (at most ``row_block`` rows at a time
 so N = 16k fits in RAM; row blocking does not change any value, each row is
@@ -48,7 +51,8 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["attention_ref", "attention_ref_rows", "attention_probs", "attention_ref_rect"]
+__all__ = ["attention_ref", "attention_ref_rows", "attention_probs", "attention_ref_rect", "attention_bwd_ref",
+           "attention_bwd_ref_rows"]
 
 
 def _as_f64(x) -> np.ndarray:
@@ -194,3 +198,91 @@ def attention_ref_rect(q, k, v, causal: bool = False, scale: float | None = None
                 o[b, h, rows] = ob
                 lse[b, h, rows] = lb
     return o, lse
+
+
+# ---------------------------------------------------------------------- backward
+#
+# Gradients of the same definition for an upstream gradient dO (the pages say
+# only that gradient comparisons use tolerances -- iplexlaw blog, "Tiling
+# preserves the attention calculation" -- so the definition is the chain rule
+# through the three steps above, written out):
+#
+#     dV     = P^T dO
+#     dP     = dO V^T
+#     dS_ij  = P_ij (dP_ij - sum_k P_ik dP_ik)       (softmax Jacobian, per row)
+#     dQ     = scale * dS K
+#     dK     = scale * dS^T Q
+#
+# Masked entries have P_ij = 0, hence dS_ij = 0.  The row sum
+# sum_k P_ik dP_ik is taken from P and dP as written (not from O).
+
+def _probs_one_head(q, k, causal, scale, offset=0):
+    """The materialised P [Nq, Nk] of one head (rows with no key: zeros)."""
+    rows = np.arange(q.shape[0])
+    s = np.where(_allowed_mask(rows, k.shape[0], causal, offset), scale * (q @ k.T), -np.inf)
+    m = np.max(s, axis=1, keepdims=True)
+    empty = ~np.isfinite(m)
+    e = np.exp(s - np.where(empty, 0.0, m))
+    l = np.sum(e, axis=1, keepdims=True)
+    return np.where(empty, 0.0, e / np.where(empty, 1.0, l))
+
+
+def _bwd_one_head(q, k, v, do, causal, scale):
+    p = _probs_one_head(q, k, causal, scale)
+    dv = p.T @ do
+    dp = do @ v.T
+    ds = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+    return scale * (ds @ k), scale * (ds.T @ q), dv
+
+
+def attention_bwd_ref(q, k, v, do, causal: bool = False, scale: float | None = None):
+    """Exact gradients (dQ, dK, dV) of attention for [B, H, N, d] inputs and dO.
+
+    Float64 throughout; the full N x N probability matrix of each head is
+    materialised (test sizes only).
+    """
+    q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape or do.shape != q.shape:
+        raise ValueError("q, k, v, do must share the shape [B, H, N, d]")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    for b in range(B):
+        for h in range(H):
+            dq[b, h], dk[b, h], dv[b, h] = _bwd_one_head(q[b, h], k[b, h], v[b, h], do[b, h], causal, float(scale))
+    return dq, dk, dv
+
+
+def attention_bwd_ref_rows(q, k, v, do, b: int, h: int, rows, causal: bool = False, scale: float | None = None,
+                           row_block: int = 1024):
+    """dQ, dK and dV rows ``rows`` of head (b, h), for long sequences.
+
+    dQ row i needs row i of P and dP; dK and dV row j need column j of P and
+    dS, i.e. every query row, which is processed ``row_block`` rows at a time
+    (blocking over query rows changes no value: each row is computed from all
+    of its keys at once, and column sums are plain sums over rows).
+    Returns (dQ [R, d], dK [R, d], dV [R, d]) float64.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    qb, kb, vb, dob = (np.asarray(t[b, h], dtype=np.float64) for t in (q, k, v, do))
+    N, d = qb.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    scale = float(scale)
+    dk = np.zeros((rows.size, d))
+    dv = np.zeros((rows.size, d))
+    dq = np.zeros((rows.size, d))
+    for r0 in range(0, N, row_block):
+        qr = np.arange(r0, min(N, r0 + row_block))
+        s = np.where(_allowed_mask(qr, N, causal), scale * (qb[qr] @ kb.T), -np.inf)
+        m = np.max(s, axis=1, keepdims=True)
+        e = np.exp(s - m)
+        p = e / np.sum(e, axis=1, keepdims=True)
+        dp = dob[qr] @ vb.T
+        ds = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+        dv += p[:, rows].T @ dob[qr]
+        dk += scale * (ds[:, rows].T @ qb[qr])
+        sel = (rows >= r0) & (rows < r0 + qr.size)
+        dq[sel] = scale * (ds[rows[sel] - r0] @ kb)
+    return dq, dk, dv
