@@ -2,12 +2,13 @@
 
 ``fwd(q, k, v, causal, scale) -> (O, LSE)`` runs the tiled, online-softmax
 forward, and ``fwd_splitkv`` the same operation for few queries against many
-keys (decoding) with the keys split over CTAs, in the hand-written CUDA kernels of ``libfa2.so`` (C ABI declared in
+keys (decoding) with the keys split over CTAs, and ``bwd`` the gradients, in the hand-written CUDA kernels of ``libfa2.so`` (C ABI declared in
 ``include/fa2.h``).  The library is loaded on first use; nothing here falls
 back to another implementation.
 """
-from .binding import (EXPORTS, FA2Error, fwd, fwd_host, fwd_inject_timeout, fwd_splitkv, load,  # noqa: F401
-                      splitkv_splits, splitkv_workspace_bytes, sync_status, workspace_bytes)
+from .binding import (EXPORTS, FA2Error, bwd, bwd_workspace_bytes, fwd, fwd_host, fwd_inject_timeout,  # noqa: F401
+                      fwd_splitkv, load, splitkv_splits, splitkv_workspace_bytes, sync_status, workspace_bytes)
 
-__all__ = ["fwd", "fwd_host", "fwd_inject_timeout", "fwd_splitkv", "load", "splitkv_splits",
+__all__ = ["fwd", "bwd", "bwd_workspace_bytes", "fwd_host", "fwd_inject_timeout", "fwd_splitkv", "load",
+           "splitkv_splits",
            "splitkv_workspace_bytes", "sync_status", "workspace_bytes", "FA2Error", "EXPORTS"]

@@ -22,8 +22,8 @@ FA2_OK, FA2_ERR_INVALID_ARG, FA2_ERR_UNSUPPORTED, FA2_ERR_CUDA, FA2_ERR_TIMEOUT 
 #: Every symbol the header declares.
 EXPORTS = ("fa2_fwd", "fa2_fwd_host", "fa2_fwd_host_workspace_bytes", "fa2_sync_status",
            "fa2_fwd_inject_timeout", "fa2_fwd_splitkv", "fa2_fwd_splitkv_splits",
-           "fa2_fwd_splitkv_workspace_bytes", "fa2_fwd_splitkv_static", "fa2_strerror", "fa2_last_error_detail",
-           "fa2_version")
+           "fa2_fwd_splitkv_workspace_bytes", "fa2_fwd_splitkv_static", "fa2_bwd", "fa2_bwd_workspace_bytes",
+           "fa2_strerror", "fa2_last_error_detail", "fa2_version")
 
 _lib = None
 
@@ -59,6 +59,10 @@ def load() -> ctypes.CDLL:
     lib.fa2_fwd_splitkv_static.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _float,
                                            _int, _vp]
     lib.fa2_fwd_splitkv_static.restype = _int
+    lib.fa2_bwd.argtypes = [_vp] * 9 + [_int] * 5 + [_float, _vp, ctypes.c_size_t, _vp]
+    lib.fa2_bwd.restype = _int
+    lib.fa2_bwd_workspace_bytes.argtypes = [_int] * 4
+    lib.fa2_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.fa2_strerror.argtypes = [_int]
     lib.fa2_strerror.restype = ctypes.c_char_p
     lib.fa2_last_error_detail.argtypes = []
@@ -271,3 +275,39 @@ def fwd_splitkv_static(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal
                                     _stream_handle(stream))
     _check(st, lib)
     return out, lse
+
+
+def bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(load().fa2_bwd_workspace_bytes(B, H, N, d))
+
+
+def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor,
+        causal: bool = False, scale: float | None = None, dq: torch.Tensor | None = None,
+        dk: torch.Tensor | None = None, dv: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+        stream=None):
+    """Gradients (dQ, dK, dV) of exact attention on CUDA tensors.
+
+    ``o`` and ``lse`` are the forward's outputs for the same q, k, v, causal
+    and scale; ``dout`` is the upstream gradient of O.  Asynchronous on
+    ``stream``.  ``workspace`` is an optional uint8 CUDA tensor of at least
+    :func:`bwd_workspace_bytes` bytes, 256-byte aligned.
+    """
+    lib = load()
+    _check_qkv(q, k, v, "cuda")
+    _check_qkv(o, dout, q, "cuda")
+    B, H, N, d = q.shape
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, N] tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = bwd_workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    st = lib.fa2_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                     dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                     workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+    _check(st, lib)
+    return dq, dk, dv

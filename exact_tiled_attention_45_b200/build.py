@@ -19,6 +19,7 @@ LIB_NAME = "libfa2.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 SOURCES = [os.path.join(CSRC, "fa2_fwd.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, "sm100_ptx.cuh"), os.path.join(CSRC, "fa2_splitkv.cuh"),
+                  os.path.join(CSRC, "fa2_bwd.cuh"),
                   os.path.join(INCLUDE, "fa2.h")]
 
 NVCC_FLAGS = [

@@ -1,0 +1,625 @@
+// Backward pass of exact attention.  Included by fa2_fwd.cu inside
+// namespace fa2 (one translation unit: shares the status word and helpers).
+//
+// Given Q, K, V, the forward output O, its per-row logsumexp LSE and the
+// upstream gradient dO, with P = exp(scale * Q K^T - LSE) (masked entries 0):
+//     D_i = sum_k dO_ik O_ik          (= sum_j P_ij dP_ij, since O = P V)
+//     dV  = P^T dO
+//     dP  = dO V^T
+//     dS  = P o (dP - D)              (o: elementwise; D broadcast along rows)
+//     dQ  = scale * dS K
+//     dK  = scale * dS^T Q
+// The pages state only that gradients are compared with tolerances (iplexlaw
+// blog "FlashAttention-2: making long-context attention run efficiently on
+// GPUs", section "Tiling preserves the attention calculation"); the formulas
+// are the chain rule through the forward definition, and the forward LSE is
+// what lets P be recomputed tile by tile without a second softmax pass.
+//
+// Two kernels, no atomics.  Each keeps one 128-row tile resident and streams
+// the other operand's tiles, with P and dS recomputed per tile pair:
+//   fa2_bwd_dq_kernel    one CTA per query tile: S = Q K_j^T, dP = dO V_j^T,
+//                        dQ += dS K_j (3 MMAs per key tile); it also writes
+//                        lse2 = LSE * log2(e) and D per row to the workspace;
+//   fa2_bwd_dkdv_kernel  one CTA per key tile: S^T = K Q_i^T, dP^T = V dO_i^T,
+//                        dV += P^T dO_i, dK += dS^T Q_i (4 MMAs per query tile).
+// Seven MMAs per tile pair instead of five: dQ is not accumulated across CTAs.
+//
+// Roles (192 threads): warps 0-3 elementwise (thread r <-> tile row r <->
+// TMEM lane r), warp 4 TMA producer, warp 5 MMA issuer.  P (dK/dV kernel) and
+// dS are packed to bf16 over the first 64 columns of their score tile in
+// TMEM and read from there by the next MMA.  Every wait is bounded.
+
+constexpr int BWD_THREADS = 192;
+constexpr int BWD_PRODUCER_WARP = 4;
+constexpr int BWD_MMA_WARP = 5;
+constexpr float LOG2E_F = 1.4426950408889634f;
+
+template <int HD>
+struct BwdCfg {
+  static constexpr int KCH = HD / 64;
+  static constexpr int CHUNK_BYTES = 128 * 128;
+  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;
+  // dQ kernel: Q and dO resident, K and V rings.
+  static constexpr int DQ_KS = (HD == 128) ? 3 : 4;
+  static constexpr int DQ_VS = (HD == 128) ? 2 : 4;
+  static constexpr int DQ_OFF_Q = 0;
+  static constexpr int DQ_OFF_DO = DQ_OFF_Q + TILE_BYTES;
+  static constexpr int DQ_OFF_K = DQ_OFF_DO + TILE_BYTES;
+  static constexpr int DQ_OFF_V = DQ_OFF_K + DQ_KS * TILE_BYTES;
+  static constexpr int DQ_OFF_BAR = DQ_OFF_V + DQ_VS * TILE_BYTES;
+  static constexpr int DQ_SMEM = DQ_OFF_BAR + 256 + 1024;
+  // dK/dV kernel: K and V resident, a ring of (Q_i, dO_i, lse2_i, D_i).
+  static constexpr int KV_QS = (HD == 128) ? 2 : 3;
+  static constexpr int KV_OFF_K = 0;
+  static constexpr int KV_OFF_V = TILE_BYTES;
+  static constexpr int KV_OFF_Q = 2 * TILE_BYTES;
+  static constexpr int KV_OFF_DO = KV_OFF_Q + KV_QS * TILE_BYTES;
+  static constexpr int KV_OFF_VEC = KV_OFF_DO + KV_QS * TILE_BYTES;  // per stage: lse2[128], D[128]
+  static constexpr int KV_OFF_BAR = KV_OFF_VEC + KV_QS * 1024;
+  static constexpr int KV_SMEM = KV_OFF_BAR + 256 + 1024;
+  static_assert(DQ_SMEM <= 232448 && KV_SMEM <= 232448, "shared memory budget");
+};
+
+struct BwdParams {
+  const __nv_bfloat16* o;     // forward output [B*H, N, d]
+  const __nv_bfloat16* dout;  // upstream gradient [B*H, N, d]
+  const float* lse;           // forward logsumexp (natural log) [B*H, N]
+  float* lse2;                // workspace [B*H, n_tiles*128]: LSE * log2(e); +inf past N
+  float* dvec;                // workspace [B*H, n_tiles*128]: D; 0 past N
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  int N;
+  int BH;
+  int n_tiles;      // ceil(N / 128), for queries and keys alike
+  int group_heads;  // heads per launch-order group
+  float scale;
+  float scale_log2;
+  unsigned long long timeout_ns;
+};
+
+// Work item of a 1-D grid: heads in groups of group_heads, tile rank the slow
+// index inside a group; with causal masking rank 0 is the heaviest tile (the
+// last query tile for dQ, the first key tile for dK/dV).
+template <bool CAUSAL, bool HEAVY_IS_LAST>
+__device__ __forceinline__ void bwd_item(const BwdParams& p, int& bh, int& tile) {
+  const int per_group = p.group_heads * p.n_tiles;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int in_grp = static_cast<int>(blockIdx.x) - grp * per_group;
+  const int grp_heads = min(p.group_heads, p.BH - grp * p.group_heads);
+  const int rank = in_grp / grp_heads;
+  bh = grp * p.group_heads + (in_grp - rank * grp_heads);
+  tile = (CAUSAL && HEAVY_IS_LAST) ? (p.n_tiles - 1 - rank) : rank;
+}
+
+// Row-major bf16 row store of 32 fp32 accumulator columns (times f).
+__device__ __forceinline__ void store_row32_bf16(__nv_bfloat16* dst, const uint32_t (&a)[32], float f) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int e = 0; e < 32; e += 8)
+    d4[e / 8] = make_uint4(pack_bf16x2(__uint_as_float(a[e]) * f, __uint_as_float(a[e + 1]) * f),
+                           pack_bf16x2(__uint_as_float(a[e + 2]) * f, __uint_as_float(a[e + 3]) * f),
+                           pack_bf16x2(__uint_as_float(a[e + 4]) * f, __uint_as_float(a[e + 5]) * f),
+                           pack_bf16x2(__uint_as_float(a[e + 6]) * f, __uint_as_float(a[e + 7]) * f));
+}
+
+// dS for 128 keys of one row: reads dP from TMEM 32 columns at a time and
+// writes dS (bf16 pairs) over the first 64 columns.  Chunk q writes packed
+// columns [16q, 16q+16), which held dP of keys 16q..16q+15: chunk q/2 <= q
+// has already read them.
+__device__ __forceinline__ void ds_to_tmem(uint32_t dp_addr, const float (&p)[128], const float* dsub, bool per_col,
+                                           float dsub_row) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t dp[32];
+    tmem_ld32(dp_addr + 32 * q, dp);
+    tmem_wait_ld();
+    reg_fence32(dp);
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int c0 = 32 * q + 2 * e;
+      const float d0 = per_col ? dsub[c0] : dsub_row;
+      const float d1 = per_col ? dsub[c0 + 1] : dsub_row;
+      pk[e] = pack_bf16x2(p[c0] * (__uint_as_float(dp[2 * e]) - d0), p[c0 + 1] * (__uint_as_float(dp[2 * e + 1]) - d1));
+    }
+    tmem_st16(dp_addr + 16 * q, pk);
+  }
+}
+
+struct DqBars {
+  uint64_t qdo_full;
+  uint64_t k_full[4], k_empty[4];
+  uint64_t v_full[4], v_empty[4];
+  uint64_t s_full, s_free, dp_full, ds_ready, mma_final;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(DqBars) <= 256, "barrier block");
+
+// TMEM columns of the dQ kernel: S [0,128), dP [128,256), dQ [256, 256+d).
+constexpr uint32_t BQ_S = 0, BQ_DP = 128, BQ_DQ = 256;
+
+template <int HD, bool CAUSAL>
+__global__ void __launch_bounds__(BWD_THREADS, 1)
+    fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                      const BwdParams p) {
+  using C = BwdCfg<HD>;
+  int bh, qt;
+  bwd_item<CAUSAL, true>(p, bh, qt);
+  const int q0 = qt * BM;
+  const int nkv = CAUSAL ? min(qt + 1, p.n_tiles) : p.n_tiles;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+  DqBars* bars = reinterpret_cast<DqBars*>(smem + C::DQ_OFF_BAR);
+  volatile int* abort_flag = &bars->abort;
+  const uint32_t sQ = base + C::DQ_OFF_Q, sDO = base + C::DQ_OFF_DO;
+  const uint32_t sK = base + C::DQ_OFF_K, sV = base + C::DQ_OFF_V;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->qdo_full), 1);
+    for (int s = 0; s < C::DQ_KS; ++s) {
+      mbar_init(smem_u32(&bars->k_full[s]), 1);
+      mbar_init(smem_u32(&bars->k_empty[s]), 1);
+    }
+    for (int s = 0; s < C::DQ_VS; ++s) {
+      mbar_init(smem_u32(&bars->v_full[s]), 1);
+      mbar_init(smem_u32(&bars->v_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bars->s_full), 1);
+    mbar_init(smem_u32(&bars->s_free), 4);
+    mbar_init(smem_u32(&bars->dp_full), 1);
+    mbar_init(smem_u32(&bars->ds_ready), 4);
+    mbar_init(smem_u32(&bars->mma_final), 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == BWD_MMA_WARP) {
+    tmem_alloc(smem_u32(&bars->tmem_base), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == BWD_PRODUCER_WARP && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const unsigned long long to = p.timeout_ns;
+
+  if (warp == BWD_PRODUCER_WARP) {
+    if (lane == 0) {
+      const uint32_t bq = smem_u32(&bars->qdo_full);
+      mbar_arrive_expect_tx(bq, 2 * C::TILE_BYTES);
+      for (int c = 0; c < C::KCH; ++c) {
+        tma_load_3d(sQ + c * C::CHUNK_BYTES, &tm_q, bq, c * 64, q0, bh);
+        tma_load_3d(sDO + c * C::CHUNK_BYTES, &tm_do, bq, c * 64, q0, bh);
+      }
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < nkv; ++j) {
+        const int ks = j % C::DQ_KS, vs = j % C::DQ_VS;
+        if (j >= C::DQ_KS &&
+            !wait_bounded(smem_u32(&bars->k_empty[ks]), ((j / C::DQ_KS) - 1) & 1, abort_flag, to, ROLE_PRODUCER))
+          break;
+        const uint32_t kb = smem_u32(&bars->k_full[ks]);
+        mbar_arrive_expect_tx(kb, C::TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sK + ks * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_k, kb, c * 64, j * BN, bh);
+        ++k_issued;
+        if (j >= C::DQ_VS &&
+            !wait_bounded(smem_u32(&bars->v_empty[vs]), ((j / C::DQ_VS) - 1) & 1, abort_flag, to, ROLE_PRODUCER))
+          break;
+        const uint32_t vb = smem_u32(&bars->v_full[vs]);
+        mbar_arrive_expect_tx(vb, C::TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sV + vs * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_v, vb, c * 64, j * BN, bh);
+        ++v_issued;
+      }
+      wait_drain(bq, 0, to);
+      for (int x = (k_issued > C::DQ_KS ? k_issued - C::DQ_KS : 0); x < k_issued; ++x)
+        wait_drain(smem_u32(&bars->k_full[x % C::DQ_KS]), (x / C::DQ_KS) & 1, to);
+      for (int x = (v_issued > C::DQ_VS ? v_issued - C::DQ_VS : 0); x < v_issued; ++x)
+        wait_drain(smem_u32(&bars->v_full[x % C::DQ_VS]), (x / C::DQ_VS) & 1, to);
+    }
+  } else if (warp == BWD_MMA_WARP) {
+    // S(0), dP(0); then per j >= 1: S(j), dQ(j-1), dP(j).  dS(j-1) lives in
+    // dP's columns, so dP(j) is issued after dQ(j-1) has been (in order).
+    if (lane == 0) {
+      constexpr uint32_t IDESC_SS = idesc_bf16_f32(BM, BN, false, false);
+      constexpr uint32_t IDESC_DQ = idesc_bf16_f32(BM, HD, false, true);
+      auto mma_kmajor = [&](uint32_t d_tmem, uint32_t a, uint32_t b) {
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+          mma_ss(d_tmem, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b + off, 16, 1024), IDESC_SS,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = wait_bounded(smem_u32(&bars->qdo_full), 0, abort_flag, to, ROLE_MMA);
+      ok = ok && wait_bounded(smem_u32(&bars->k_full[0]), 0, abort_flag, to, ROLE_MMA);
+      if (ok) {
+        tc_fence_after();
+        mma_kmajor(tmem + BQ_S, sQ, sK);
+        mma_commit(smem_u32(&bars->s_full));
+      }
+      ok = ok && wait_bounded(smem_u32(&bars->v_full[0]), 0, abort_flag, to, ROLE_MMA);
+      if (ok) {
+        tc_fence_after();
+        mma_kmajor(tmem + BQ_DP, sDO, sV);
+        mma_commit(smem_u32(&bars->dp_full));
+        mma_commit(smem_u32(&bars->v_empty[0]));
+      }
+      for (int j = 1; ok && j <= nkv; ++j) {
+        const int i = j - 1;
+        if (j < nkv) {
+          const int ks = j % C::DQ_KS;
+          ok = wait_bounded(smem_u32(&bars->k_full[ks]), (j / C::DQ_KS) & 1, abort_flag, to, ROLE_MMA) &&
+               wait_bounded(smem_u32(&bars->s_free), i & 1, abort_flag, to, ROLE_MMA);
+          if (!ok) break;
+          tc_fence_after();
+          mma_kmajor(tmem + BQ_S, sQ, sK + ks * C::TILE_BYTES);
+          mma_commit(smem_u32(&bars->s_full));
+        }
+        ok = wait_bounded(smem_u32(&bars->ds_ready), i & 1, abort_flag, to, ROLE_MMA);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kbase = sK + (i % C::DQ_KS) * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(tmem + BQ_DQ, tmem + BQ_DP + kk * 8, smem_desc_sw128(kbase + kk * 2048, C::CHUNK_BYTES, 1024),
+                 IDESC_DQ, (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(smem_u32(&bars->k_empty[i % C::DQ_KS]));
+        if (j < nkv) {
+          const int vs = j % C::DQ_VS;
+          ok = wait_bounded(smem_u32(&bars->v_full[vs]), (j / C::DQ_VS) & 1, abort_flag, to, ROLE_MMA);
+          if (!ok) break;
+          tc_fence_after();
+          mma_kmajor(tmem + BQ_DP, sDO, sV + vs * C::TILE_BYTES);
+          mma_commit(smem_u32(&bars->dp_full));
+          mma_commit(smem_u32(&bars->v_empty[vs]));
+        }
+      }
+      mma_commit(smem_u32(&bars->mma_final));
+      wait_drain(smem_u32(&bars->mma_final), 0, to);
+    }
+  } else {
+    // ------------------------------------------------------------ elementwise warps 0..3
+    const int r = threadIdx.x;
+    const int row = q0 + r;
+    const bool valid = row < p.N;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    // D = dO . O and lse2 of this row, kept in registers and written to the
+    // workspace for the dK/dV kernel (padding rows: D = 0, lse2 = +inf).
+    float dsum = 0.f, lse2 = INFINITY;
+    if (valid) {
+      const size_t off = (static_cast<size_t>(bh) * p.N + row) * HD;
+      const uint4* o4 = reinterpret_cast<const uint4*>(p.o + off);
+      const uint4* g4 = reinterpret_cast<const uint4*>(p.dout + off);
+#pragma unroll 4
+      for (int c = 0; c < HD / 8; ++c) {
+        const uint4 a = o4[c], g = g4[c];
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          dsum = fmaf(__uint_as_float(aw[e] << 16), __uint_as_float(gw[e] << 16), dsum);
+          dsum = fmaf(__uint_as_float(aw[e] & 0xffff0000u), __uint_as_float(gw[e] & 0xffff0000u), dsum);
+        }
+      }
+      lse2 = p.lse[static_cast<size_t>(bh) * p.N + row] * LOG2E_F;
+    }
+    const size_t vrow = static_cast<size_t>(bh) * p.n_tiles * BM + q0 + r;
+    p.dvec[vrow] = dsum;
+    p.lse2[vrow] = lse2;
+
+    const float c = p.scale_log2;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      ok = wait_warp(smem_u32(&bars->s_full), j & 1, abort_flag, to);
+      if (!ok) break;
+      tc_fence_after();
+      float pr[128];
+      {
+        uint32_t s[128];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          tmem_ld32(lane_addr + BQ_S + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->s_free));
+        const int kv0 = j * BN;
+        const bool diag = CAUSAL && (j == qt);
+        const bool tail = !CAUSAL && (kv0 + BN > p.N);
+        const int lim = diag ? (row - kv0) : (p.N - 1 - kv0);  // last allowed key column
+#pragma unroll
+        for (int e = 0; e < 128; ++e) {
+          const float x = (diag || tail) && e > lim ? -INFINITY : __uint_as_float(s[e]);
+          pr[e] = ex2(x * c - lse2);
+        }
+      }
+      ok = wait_warp(smem_u32(&bars->dp_full), j & 1, abort_flag, to);
+      if (!ok) break;
+      tc_fence_after();
+      ds_to_tmem(lane_addr + BQ_DP, pr, nullptr, false, dsum);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->ds_ready));
+    }
+    if (ok) ok = wait_warp(smem_u32(&bars->mma_final), 0, abort_flag, to);
+    if (ok) {
+      tc_fence_after();
+      uint32_t a[HD / 32][32];
+#pragma unroll
+      for (int cc = 0; cc < HD / 32; ++cc) tmem_ld32(lane_addr + BQ_DQ + cc * 32, a[cc]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int cc = 0; cc < HD / 32; ++cc) reg_fence32(a[cc]);
+      if (valid) {
+        __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bh) * p.N + row) * HD;
+#pragma unroll
+        for (int cc = 0; cc < HD / 32; ++cc) store_row32_bf16(dst + cc * 32, a[cc], p.scale);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == BWD_MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+struct KvBars {
+  uint64_t kv_full;
+  uint64_t q_full[3], q_empty[3];
+  uint64_t s_full, dp_full, p_ready, ds_ready, mma_final;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(KvBars) <= 256, "barrier block");
+
+// TMEM columns of the dK/dV kernel: S^T [0,128), dP^T [128,256),
+// dV [256, 256+d), dK [256+d, 256+2d).
+constexpr uint32_t BK_S = 0, BK_DP = 128, BK_DV = 256;
+
+template <int HD, bool CAUSAL>
+__global__ void __launch_bounds__(BWD_THREADS, 1)
+    fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                        const BwdParams p) {
+  using C = BwdCfg<HD>;
+  constexpr uint32_t BK_DK = BK_DV + HD;
+  int bh, kt;
+  bwd_item<CAUSAL, false>(p, bh, kt);
+  const int k0 = kt * BN;
+  const int i_begin = CAUSAL ? kt : 0;  // query tiles that see this key tile
+  const int nq = p.n_tiles - i_begin;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+  KvBars* bars = reinterpret_cast<KvBars*>(smem + C::KV_OFF_BAR);
+  volatile int* abort_flag = &bars->abort;
+  const uint32_t sK = base + C::KV_OFF_K, sV = base + C::KV_OFF_V;
+  const uint32_t sQ = base + C::KV_OFF_Q, sDO = base + C::KV_OFF_DO;
+  const float* vec = reinterpret_cast<const float*>(smem + C::KV_OFF_VEC);
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->kv_full), 1);
+    for (int s = 0; s < C::KV_QS; ++s) {
+      mbar_init(smem_u32(&bars->q_full[s]), 1);
+      mbar_init(smem_u32(&bars->q_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bars->s_full), 1);
+    mbar_init(smem_u32(&bars->dp_full), 1);
+    mbar_init(smem_u32(&bars->p_ready), 4);
+    mbar_init(smem_u32(&bars->ds_ready), 4);
+    mbar_init(smem_u32(&bars->mma_final), 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == BWD_MMA_WARP) {
+    tmem_alloc(smem_u32(&bars->tmem_base), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == BWD_PRODUCER_WARP && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const unsigned long long to = p.timeout_ns;
+  const size_t vec_head = static_cast<size_t>(bh) * p.n_tiles * BM;
+
+  if (warp == BWD_PRODUCER_WARP) {
+    if (lane == 0) {
+      const uint32_t bkv = smem_u32(&bars->kv_full);
+      mbar_arrive_expect_tx(bkv, 2 * C::TILE_BYTES);
+      for (int c = 0; c < C::KCH; ++c) {
+        tma_load_3d(sK + c * C::CHUNK_BYTES, &tm_k, bkv, c * 64, k0, bh);
+        tma_load_3d(sV + c * C::CHUNK_BYTES, &tm_v, bkv, c * 64, k0, bh);
+      }
+      int issued = 0;
+      for (int t = 0; t < nq; ++t) {
+        const int s = t % C::KV_QS;
+        if (t >= C::KV_QS &&
+            !wait_bounded(smem_u32(&bars->q_empty[s]), ((t / C::KV_QS) - 1) & 1, abort_flag, to, ROLE_PRODUCER))
+          break;
+        const int i = i_begin + t;
+        const uint32_t bq = smem_u32(&bars->q_full[s]);
+        mbar_arrive_expect_tx(bq, 2 * C::TILE_BYTES + 1024);
+        for (int c = 0; c < C::KCH; ++c) {
+          tma_load_3d(sQ + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, bq, c * 64, i * BM, bh);
+          tma_load_3d(sDO + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_do, bq, c * 64, i * BM, bh);
+        }
+        const uint32_t sv = base + C::KV_OFF_VEC + s * 1024;
+        bulk_load_1d(sv, p.lse2 + vec_head + i * BM, 512, bq);
+        bulk_load_1d(sv + 512, p.dvec + vec_head + i * BM, 512, bq);
+        ++issued;
+      }
+      wait_drain(bkv, 0, to);
+      for (int x = (issued > C::KV_QS ? issued - C::KV_QS : 0); x < issued; ++x)
+        wait_drain(smem_u32(&bars->q_full[x % C::KV_QS]), (x / C::KV_QS) & 1, to);
+    }
+  } else if (warp == BWD_MMA_WARP) {
+    // S^T(0), dP^T(0); then per query tile t: dV(t), S^T(t+1), dK(t),
+    // dP^T(t+1).  P^T(t) lives in S^T's columns and dS^T(t) in dP^T's, so
+    // each overwrite is issued after the MMA that reads them (in order).
+    if (lane == 0) {
+      constexpr uint32_t IDESC_SS = idesc_bf16_f32(BN, BM, false, false);
+      constexpr uint32_t IDESC_ACC = idesc_bf16_f32(BN, HD, false, true);
+      auto mma_kmajor = [&](uint32_t d_tmem, uint32_t a, uint32_t b) {
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+          mma_ss(d_tmem, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b + off, 16, 1024), IDESC_SS,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      auto mma_acc = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b + kk * 2048, C::CHUNK_BYTES, 1024), IDESC_ACC,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = wait_bounded(smem_u32(&bars->kv_full), 0, abort_flag, to, ROLE_MMA) &&
+                wait_bounded(smem_u32(&bars->q_full[0]), 0, abort_flag, to, ROLE_MMA);
+      if (ok) {
+        tc_fence_after();
+        mma_kmajor(tmem + BK_S, sK, sQ);
+        mma_commit(smem_u32(&bars->s_full));
+        mma_kmajor(tmem + BK_DP, sV, sDO);
+        mma_commit(smem_u32(&bars->dp_full));
+      }
+      for (int t = 0; ok && t < nq; ++t) {
+        const int s = t % C::KV_QS;
+        ok = wait_bounded(smem_u32(&bars->p_ready), t & 1, abort_flag, to, ROLE_MMA);
+        if (!ok) break;
+        tc_fence_after();
+        mma_acc(tmem + BK_DV, tmem + BK_S, sDO + s * C::TILE_BYTES, t > 0);
+        const bool more = t + 1 < nq;
+        const int s1 = (t + 1) % C::KV_QS;
+        if (more) {
+          ok = wait_bounded(smem_u32(&bars->q_full[s1]), ((t + 1) / C::KV_QS) & 1, abort_flag, to, ROLE_MMA);
+          if (!ok) break;
+          tc_fence_after();
+          mma_kmajor(tmem + BK_S, sK, sQ + s1 * C::TILE_BYTES);
+          mma_commit(smem_u32(&bars->s_full));
+        }
+        ok = wait_bounded(smem_u32(&bars->ds_ready), t & 1, abort_flag, to, ROLE_MMA);
+        if (!ok) break;
+        tc_fence_after();
+        mma_acc(tmem + BK_DK, tmem + BK_DP, sQ + s * C::TILE_BYTES, t > 0);
+        mma_commit(smem_u32(&bars->q_empty[s]));
+        if (more) {
+          mma_kmajor(tmem + BK_DP, sV, sDO + s1 * C::TILE_BYTES);
+          mma_commit(smem_u32(&bars->dp_full));
+        }
+      }
+      mma_commit(smem_u32(&bars->mma_final));
+      wait_drain(smem_u32(&bars->mma_final), 0, to);
+    }
+  } else {
+    // ------------------------------------------------------------ elementwise warps 0..3
+    const int r = threadIdx.x;
+    const int key = k0 + r;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float c = p.scale_log2;
+    bool ok = true;
+    for (int t = 0; t < nq; ++t) {
+      const int s = t % C::KV_QS;
+      const int i = i_begin + t;
+      ok = wait_warp(smem_u32(&bars->s_full), t & 1, abort_flag, to) &&
+           wait_warp(smem_u32(&bars->q_full[s]), (t / C::KV_QS) & 1, abort_flag, to);
+      if (!ok) break;
+      tc_fence_after();
+      const float* l2 = vec + s * 256;  // lse2 of the tile's 128 queries (+inf past N)
+      const float* dd = l2 + 128;       // D of the tile's 128 queries
+      float pr[128];
+      {
+        uint32_t sv[128];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          tmem_ld32(lane_addr + BK_S + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
+        const bool diag = CAUSAL && (i == kt);  // query 128i + e sees this key only if e >= r
+#pragma unroll
+        for (int e = 0; e < 128; ++e) {
+          const float x = (diag && e < r) ? -INFINITY : __uint_as_float(sv[e]);
+          pr[e] = ex2(x * c - l2[e]);
+        }
+      }
+      // P^T (bf16) over the first 64 score columns, for dV += P^T dO.
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pr[64 * h + 2 * e], pr[64 * h + 2 * e + 1]);
+        tmem_st32(lane_addr + BK_S + 32 * h, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready));
+      ok = wait_warp(smem_u32(&bars->dp_full), t & 1, abort_flag, to);
+      if (!ok) break;
+      tc_fence_after();
+      ds_to_tmem(lane_addr + BK_DP, pr, dd, true, 0.f);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->ds_ready));
+    }
+    if (ok) ok = wait_warp(smem_u32(&bars->mma_final), 0, abort_flag, to);
+    if (ok) {
+      tc_fence_after();
+      const bool valid = key < p.N;
+      const size_t off = (static_cast<size_t>(bh) * p.N + key) * HD;
+#pragma unroll
+      for (int cc = 0; cc < HD / 32; ++cc) {
+        uint32_t a[32];
+        tmem_ld32(lane_addr + BK_DV + cc * 32, a);
+        tmem_wait_ld();
+        reg_fence32(a);
+        if (valid) store_row32_bf16(p.dv + off + cc * 32, a, 1.f);
+      }
+#pragma unroll
+      for (int cc = 0; cc < HD / 32; ++cc) {
+        uint32_t a[32];
+        tmem_ld32(lane_addr + BK_DK + cc * 32, a);
+        tmem_wait_ld();
+        reg_fence32(a);
+        if (valid) store_row32_bf16(p.dk + off + cc * 32, a, p.scale);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == BWD_MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}

@@ -625,6 +625,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 #include "fa2_splitkv.cuh"
+#include "fa2_bwd.cuh"
 
 // ====================================================================== host
 
@@ -944,6 +945,133 @@ static int splitkv_impl(const void* q, const void* k, const void* v, void* o, fl
                 : skv_launch_t<128, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
 }
 
+// ------------------------------------------------------------------ backward host side
+
+// Workspace of the backward: lse2 then D, fp32 [B*H, ceil(N/128)*128] each,
+// each starting on a 256-byte boundary.
+static size_t bwd_workspace_bytes_for(int B, int H, int N) {
+  const size_t rows = static_cast<size_t>(B) * H * static_cast<size_t>((N + BM - 1) / BM) * BM;
+  return 2 * round256(rows * 4);
+}
+
+template <int HD, bool CAUSAL>
+static int bwd_launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                        const BwdParams& prm, cudaStream_t stream) {
+  using C = BwdCfg<HD>;
+  static int attr_done_mask = 0;  // per device bit (devices 0..31)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    set_detail("cudaGetDevice failed");
+    return FA2_ERR_CUDA;
+  }
+  auto kq = fa2_bwd_dq_kernel<HD, CAUSAL>;
+  auto kkv = fa2_bwd_dkdv_kernel<HD, CAUSAL>;
+  if (dev >= 32 || !(attr_done_mask & (1 << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::DQ_SMEM);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, C::KV_SMEM);
+    if (e != cudaSuccess) {
+      set_detail("cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+      return FA2_ERR_CUDA;
+    }
+    if (dev < 32) attr_done_mask |= (1 << dev);
+  }
+  const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_tiles);
+  kq<<<grid, BWD_THREADS, C::DQ_SMEM, stream>>>(tq, tk, tv, tdo, prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_detail("dQ kernel launch: %s", cudaGetErrorString(e));
+    return FA2_ERR_CUDA;
+  }
+  kkv<<<grid, BWD_THREADS, C::KV_SMEM, stream>>>(tq, tk, tv, tdo, prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_detail("dK/dV kernel launch: %s", cudaGetErrorString(e));
+    return FA2_ERR_CUDA;
+  }
+  return FA2_OK;
+}
+
+static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                    void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
+                    void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  g_detail[0] = 0;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) {
+    set_detail("null pointer");
+    return FA2_ERR_INVALID_ARG;
+  }
+  if (B < 1 || H < 1 || N < 1 || B > 65535 || H > 65535 ||
+      static_cast<long long>(B) * H * ((N + BM - 1) / BM) > 0x7fffffffLL) {
+    set_detail("bad sizes B=%d H=%d N=%d (need B, H <= 65535 and B*H*ceil(N/128) < 2^31)", B, H, N);
+    return FA2_ERR_INVALID_ARG;
+  }
+  if (!std::isfinite(scale) || !(scale > 0.f)) {
+    set_detail("scale must be finite and positive");
+    return FA2_ERR_INVALID_ARG;
+  }
+  if (d != 64 && d != 128) {
+    set_detail("head dimension %d not supported (64 or 128)", d);
+    return FA2_ERR_UNSUPPORTED;
+  }
+  const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                        reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o) |
+                        reinterpret_cast<uintptr_t>(dout) | reinterpret_cast<uintptr_t>(dq) |
+                        reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv);
+  if ((mis & 15u) || (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) {
+    set_detail("misaligned pointer (tensors need 16 bytes, lse 4, workspace 256)");
+    return FA2_ERR_INVALID_ARG;
+  }
+  const size_t need = bwd_workspace_bytes_for(B, H, N);
+  if (workspace_bytes < need) {
+    set_detail("workspace too small: %zu bytes, need %zu", workspace_bytes, need);
+    return FA2_ERR_INVALID_ARG;
+  }
+  const size_t BH = static_cast<size_t>(B) * H;
+  const size_t tb = BH * N * d * 2, lb = BH * N * 4;
+  const void* ins[6] = {q, k, v, o, dout, lse};
+  const size_t in_bytes[6] = {tb, tb, tb, tb, tb, lb};
+  void* outs[4] = {dq, dk, dv, workspace};
+  const size_t out_bytes[4] = {tb, tb, tb, need};
+  for (int a = 0; a < 4; ++a) {
+    for (int b = 0; b < 6; ++b)
+      if (overlap(outs[a], out_bytes[a], ins[b], in_bytes[b])) {
+        set_detail("output or workspace buffers overlap inputs");
+        return FA2_ERR_INVALID_ARG;
+      }
+    for (int b = a + 1; b < 4; ++b)
+      if (overlap(outs[a], out_bytes[a], outs[b], out_bytes[b])) {
+        set_detail("output or workspace buffers overlap each other");
+        return FA2_ERR_INVALID_ARG;
+      }
+  }
+  CUtensorMap tq, tk, tv, tdo;
+  int st;
+  if ((st = make_tmap(&tq, q, d, N, static_cast<int>(BH))) != FA2_OK) return st;
+  if ((st = make_tmap(&tk, k, d, N, static_cast<int>(BH))) != FA2_OK) return st;
+  if ((st = make_tmap(&tv, v, d, N, static_cast<int>(BH))) != FA2_OK) return st;
+  if ((st = make_tmap(&tdo, dout, d, N, static_cast<int>(BH))) != FA2_OK) return st;
+  BwdParams prm;
+  prm.o = static_cast<const __nv_bfloat16*>(o);
+  prm.dout = static_cast<const __nv_bfloat16*>(dout);
+  prm.lse = lse;
+  prm.n_tiles = (N + BM - 1) / BM;
+  prm.lse2 = static_cast<float*>(workspace);
+  prm.dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) + need / 2);
+  prm.dq = static_cast<__nv_bfloat16*>(dq);
+  prm.dk = static_cast<__nv_bfloat16*>(dk);
+  prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.N = N;
+  prm.BH = static_cast<int>(BH);
+  prm.group_heads = causal ? causal_group_heads(static_cast<int>(BH), N, d, prm.n_tiles) : 1;
+  prm.scale = scale;
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+  prm.timeout_ns = DEFAULT_TIMEOUT_NS;
+  if (d == 64)
+    return causal ? bwd_launch_t<64, true>(tq, tk, tv, tdo, prm, stream)
+                  : bwd_launch_t<64, false>(tq, tk, tv, tdo, prm, stream);
+  return causal ? bwd_launch_t<128, true>(tq, tk, tv, tdo, prm, stream)
+                : bwd_launch_t<128, false>(tq, tk, tv, tdo, prm, stream);
+}
+
 // ------------------------------------------------------------------ split-K/V with library-owned scratch
 // For callers that cannot allocate device memory (see fa2_fwd_splitkv_static
 // in fa2.h): the partial outputs live in this fixed array instead of a
@@ -1119,6 +1247,18 @@ int fa2_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o,
   return fa2::splitkv_impl(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, n_splits, scratch,
                            scratch ? static_cast<size_t>(FA2_SPLITKV_STATIC_SCRATCH_BYTES) : 0,
                            static_cast<cudaStream_t>(stream));
+}
+
+size_t fa2_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  return fa2::bwd_workspace_bytes_for(B, H, N);
+}
+
+int fa2_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
+            void* dk, void* dv, int B, int H, int N, int d, int causal, float scale, void* workspace,
+            size_t workspace_bytes, void* stream) {
+  return fa2::bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, workspace, workspace_bytes,
+                       static_cast<cudaStream_t>(stream));
 }
 
 const char* fa2_strerror(int status) {

@@ -58,6 +58,14 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
 }
 
 // 3-D tiled bulk tensor load global -> shared, completion counted on `bar`.
+// Untiled bulk copy global -> shared (no multicast): both addresses 16-byte
+// aligned, size a multiple of 16 bytes; completes bytes on the mbarrier.
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar, int x, int y,
                                             int z) {
   asm volatile(

@@ -153,6 +153,40 @@ int fa2_fwd_splitkv_splits(int B, int H, int Nq, int Nk, int d, int n_splits);
 size_t fa2_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int n_splits);
 
 /*
+ * Backward pass of exact attention: the gradients dQ, dK, dV for an upstream
+ * gradient dO, given the forward's inputs, its output O and its LSE (iplexlaw
+ * blog "FlashAttention-2: making long-context attention run efficiently on
+ * GPUs", section "Tiling preserves the attention calculation": outputs and
+ * gradients are compared with tolerances).  With P = exp(scale*QK^T - LSE):
+ *     D = rowsum(dO o O), dV = P^T dO, dS = P o (dO V^T - D),
+ *     dQ = scale * dS K,  dK = scale * dS^T Q.
+ * P is recomputed tile by tile from LSE; the N x N matrices never reach
+ * device memory.
+ *
+ *   q, k, v, o, dout : device pointers, bf16 [B,H,N,d], contiguous,
+ *                      16-byte aligned (o and lse as written by fa2_fwd with
+ *                      the same q, k, v, causal and scale).
+ *   lse     : device pointer, fp32 [B,H,N], natural log, 4-byte aligned.
+ *   dq, dk, dv : device pointers, bf16 [B,H,N,d]; written.  They must not
+ *             overlap each other, the inputs or the workspace.
+ *   B, H, N, d, causal, scale : as for fa2_fwd (d 64 or 128; scale > 0).
+ *   workspace, workspace_bytes : caller-owned device buffer, 256-byte
+ *             aligned, of at least fa2_bwd_workspace_bytes(B,H,N,d) bytes;
+ *             it carries per-row LSE*log2(e) and rowsum(dO o O) from the
+ *             first kernel to the second.  Concurrent calls need separate
+ *             workspaces.
+ *   stream  : cudaStream_t as void*; two kernels are queued on it.
+ * Argument errors are reported before anything is launched; kernel-side
+ * timeouts through fa2_sync_status.
+ */
+int fa2_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
+            void* dk, void* dv, int B, int H, int N, int d, int causal, float scale, void* workspace,
+            size_t workspace_bytes, void* stream);
+
+/* Workspace bytes fa2_bwd needs for this shape (0 on bad sizes). */
+size_t fa2_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
  * fa2_fwd_splitkv without a workspace argument, for callers that cannot
  * allocate device memory: a plug-in running inside a host application whose
  * memory pool owns the whole device (a serving process or a framework's

@@ -201,3 +201,40 @@ def test_static_scratch_entry_rejects_on_the_host(lib):
     assert b"static scratch" in lib.fa2_last_error_detail()
     rc = lib.fa2_fwd_splitkv_static(0, FAKE, FAKE, FAKE, FAKE, 1, 1, 1, 128, 64, 0, 0.125, 0, None)
     assert rc == binding.FA2_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------- backward
+
+def _bwd(lib, B=1, H=2, N=200, d=128, causal=0, scale=0.088, ws=FAKE + (9 << 32), ws_bytes=1 << 20, **ptrs):
+    names = ["q", "k", "v", "o", "do", "lse", "dq", "dk", "dv"]
+    p = {n: FAKE + (i << 32) for i, n in enumerate(names)}
+    p.update(ptrs)
+    return lib.fa2_bwd(*(p[n] for n in names), B, H, N, d, causal, scale, ws, ws_bytes, None)
+
+
+def test_bwd_workspace_size(lib):
+    # lse2 and D, fp32, rows padded to 128 per head, each rounded to 256 bytes
+    assert lib.fa2_bwd_workspace_bytes(2, 3, 200, 128) == 2 * (2 * 3 * 256 * 4)
+    assert lib.fa2_bwd_workspace_bytes(1, 1, 1, 64) == 2 * 512
+    assert lib.fa2_bwd_workspace_bytes(1, 1, 0, 64) == 0
+    assert lib.fa2_bwd_workspace_bytes(1, 1, 8, 96) == 0
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=0), binding.FA2_ERR_INVALID_ARG),
+    (dict(dv=0), binding.FA2_ERR_INVALID_ARG),
+    (dict(ws=0), binding.FA2_ERR_INVALID_ARG),
+    (dict(N=0), binding.FA2_ERR_INVALID_ARG),
+    (dict(d=96), binding.FA2_ERR_UNSUPPORTED),
+    (dict(scale=0.0), binding.FA2_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), binding.FA2_ERR_INVALID_ARG),
+    (dict(ws=FAKE + (9 << 32) + 64), binding.FA2_ERR_INVALID_ARG),   # workspace not 256-aligned
+    (dict(ws_bytes=1024), binding.FA2_ERR_INVALID_ARG),              # too small (needs 4096)
+    (dict(dq=FAKE), binding.FA2_ERR_INVALID_ARG),                    # dq aliases q
+    (dict(dk=FAKE + (6 << 32)), binding.FA2_ERR_INVALID_ARG),        # dk aliases dq
+    (dict(ws=FAKE + (8 << 32)), binding.FA2_ERR_INVALID_ARG),        # workspace aliases dv
+    (dict(o=FAKE + (1 << 32) + 8), binding.FA2_ERR_INVALID_ARG),     # misaligned o
+])
+def test_bwd_bad_arguments_rejected_before_launch(lib, kw, expect):
+    assert _bwd(lib, **kw) == expect
+    assert lib.fa2_last_error_detail()
