@@ -39,9 +39,10 @@ METRIC = "attn fwd TFLOP/s (bf16, N=512–16k, d=64/128) and % of B200 dense BF1
 DEFAULT_WORKLOAD = "B8_H16_N2048_d128_causal"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_BF16_TFLOPS = 2250.0
+BWD_METRIC = "attn bwd TFLOP/s (bf16, FLOP = 2.5 x forward FLOP) and % of B200 dense BF16 peak"
 DECODE_METRIC = "split-K/V attn fwd effective HBM GB/s (Q,K,V read once, O,LSE written once)"
 KERNEL_SOURCES = ["exact_tiled_attention_45_b200/csrc/fa2_fwd.cu", "exact_tiled_attention_45_b200/csrc/sm100_ptx.cuh",
-                  "exact_tiled_attention_45_b200/csrc/fa2_splitkv.cuh"]
+                  "exact_tiled_attention_45_b200/csrc/fa2_splitkv.cuh", "exact_tiled_attention_45_b200/csrc/fa2_bwd.cuh"]
 
 
 def parse_args():
@@ -56,6 +57,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the timed oracle sample")
     ap.add_argument("--splits", type=int, default=0, help="key ranges for decode workloads (0 = library choice)")
     ap.add_argument("--no-gemm", action="store_true", help="skip the library GEMM comparator")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
+                    help="bwd: time the backward (dQ, dK, dV) instead of the forward")
     return ap.parse_args()
 
 
@@ -227,7 +230,14 @@ def run_reference(args, w):
     heads_per_step = 1
     q, k, v = workload_inputs(w, 0)
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
-    if is_decode(w):
+    bwd_pass = (not is_decode(w)) and args.pass_ == "bwd"
+    if bwd_pass:
+        from oracle import attention_bwd_ref
+        g = torch.Generator(device="cpu")
+        g.manual_seed(1000)
+        do = torch.randn(q.shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+        per_head, unit, metric, scale_u = 2.5 * w.flops / (w.B * w.H), "TFLOP/s", BWD_METRIC, 1e12
+    elif is_decode(w):
         per_head, unit, metric, scale_u = w.bytes / (w.B * w.H), "GB/s", DECODE_METRIC, 1e9
         heads_per_step = 16
     else:
@@ -236,7 +246,12 @@ def run_reference(args, w):
     def step(i):
         for t in range(heads_per_step):
             b, h = heads[(i * heads_per_step + t) % len(heads)]
-            oracle_head(w, q, k, v, b, h)
+            if bwd_pass:
+                sl = (slice(b, b + 1), slice(h, h + 1))
+                attention_bwd_ref(q[sl].double().numpy(), k[sl].double().numpy(), v[sl].double().numpy(),
+                                  do[sl].double().numpy(), causal=w.causal, scale=w.d ** -0.5)
+            else:
+                oracle_head(w, q, k, v, b, h)
 
     for i in range(args.warmup):
         step(i)
@@ -304,6 +319,149 @@ def gemm_comparator(w, dev, reps: int = 20) -> dict:
     del q, k, s, o
     torch.cuda.empty_cache()
     return out
+
+
+def run_backward(args, w):
+    """The backward (fa2_bwd, two kernels) on the workload; TFLOP/s by the
+    usual convention of 2.5 x the forward FLOP (five matmuls; the kernels
+    execute seven, since dQ is computed without atomics)."""
+    import torch
+    import torch.distributed as dist
+    import exact_tiled_attention_45_b200 as fa2
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    q_h, k_h, v_h = workload_inputs(w, shard_seed(rank))
+    g = torch.Generator(device="cpu")
+    g.manual_seed(1000 + shard_seed(rank))
+    do_h = torch.randn(q_h.shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
+    o, lse = fa2.fwd(q, k, v, causal=w.causal, stream=stream)
+    ws = torch.empty(fa2.bwd_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    in_bytes = 5 * q.numel() * 2 + lse.numel() * 4
+    out_bytes = 3 * q.numel() * 2
+    flops = 2.5 * w.flops
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev) if in_bytes <= l2_bytes else None
+
+    def call():
+        fa2.bwd(q, k, v, o, lse, do, causal=w.causal, dq=dq, dk=dk, dv=dv, workspace=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        call()
+    fa2.sync_status(stream)
+    sampler = ClockSampler(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    total_ms = 0.0
+    if flush is None:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            call()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        total_ms = ev0.elapsed_time(ev1)
+    else:
+        for _ in range(args.steps):
+            flush.zero_()
+            ev0.record(stream)
+            call()
+            ev1.record(stream)
+            ev1.synchronize()
+            total_ms += ev0.elapsed_time(ev1)
+    sampler.stop()
+    barrier()
+    fa2.sync_status(stream)
+    step_ms = total_ms / args.steps
+    max_ms = max_over_ranks(total_ms, dev) / args.steps
+    value = flops * world / (max_ms * 1e-3) / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        pinned = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)]
+        o_h, lse_h = o.cpu().pin_memory(), lse.cpu().pin_memory()
+        outs = [torch.empty_like(q_h).pin_memory() for _ in range(3)]
+        e2e_steps = max(3, min(args.steps, 10))
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                for dst, src in zip((q, k, v, do), pinned):
+                    dst.copy_(src, non_blocking=True)
+                o.copy_(o_h, non_blocking=True)
+                lse.copy_(lse_h, non_blocking=True)
+                call()
+                for dst, src in zip(outs, (dq, dk, dv)):
+                    dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), dev) / e2e_steps
+        e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes, "steps": e2e_steps,
+               "path": "torch pinned copies + fa2.bwd on one stream"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flops / (step_ms * 1e-3) / 1e12
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        from oracle import attention_bwd_ref
+        heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+        done, t0 = 0, time.perf_counter()
+        for b, h in heads:
+            sl = (slice(b, b + 1), slice(h, h + 1))
+            attention_bwd_ref(q_h[sl].double().numpy(), k_h[sl].double().numpy(), v_h[sl].double().numpy(),
+                              do_h[sl].double().numpy(), causal=w.causal, scale=w.d ** -0.5)
+            done += 1
+            if time.perf_counter() - t0 >= args.cpu_seconds:
+                break
+        dt = time.perf_counter() - t0
+        cpu = {"value": flops / (w.B * w.H) * done / dt / 1e12, "unit": "TFLOP/s", "cores": torch.get_num_threads(),
+               "kind": "oracle", "sample": f"{done} of {len(heads)} heads of {w.name}, backward (fp64 NumPy, {dt:.1f} s)"}
+    line = {
+        "metric": BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(w.as_dict(), seed="rank", scale=f"1/sqrt({w.d})", pass_="bwd",
+                       l2=("inputs larger than L2" if flush is None else "L2 flushed before every step"),
+                       parallelism=("single GPU" if world == 1 else f"{world} ranks, independent heads, no collective")),
+        "executed_tflops": 3.5 * w.flops / (step_ms * 1e-3) / 1e12,
+        "pct_of_peak": {"measured_burst": 100.0 * achieved / peak, "peaks": peak_kind},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": recorded_traffic(w.name + ":bwd", source_hash()),
+                     "peak_source": f"{peak_kind} bf16 burst",
+                     "kernel": "fa2_bwd_dq_kernel + fa2_bwd_dkdv_kernel (one step, both timed)",
+                     "src": source_hash()},
+        "clocks": sampler.summary(),
+        "gpu_launches": 2 * args.steps,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
 
 
 def run_decode(args, w):
@@ -465,6 +623,8 @@ def main():
         raise SystemExit("need --steps >= 1 and --warmup >= 3")
     if is_decode(w):
         return run_decode(args, w)
+    if args.pass_ == "bwd":
+        return run_backward(args, w)
 
     import torch
     import torch.distributed as dist
