@@ -70,6 +70,7 @@ struct BwdParams {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int N;
+  int d;            // head dimension of the tensors (<= HD; the kernel's tiles are zero-padded to HD)
   int BH;
   int n_tiles;      // ceil(N / 128), for queries and keys alike
   int group_heads;  // heads per launch-order group
@@ -301,11 +302,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     // workspace for the dK/dV kernel (padding rows: D = 0, lse2 = +inf).
     float dsum = 0.f, lse2 = INFINITY;
     if (valid) {
-      const size_t off = (static_cast<size_t>(bh) * p.N + row) * HD;
+      const size_t off = (static_cast<size_t>(bh) * p.N + row) * p.d;
       const uint4* o4 = reinterpret_cast<const uint4*>(p.o + off);
       const uint4* g4 = reinterpret_cast<const uint4*>(p.dout + off);
 #pragma unroll 4
-      for (int c = 0; c < HD / 8; ++c) {
+      for (int c = 0; c < p.d / 8; ++c) {
         const uint4 a = o4[c], g = g4[c];
         const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
@@ -339,9 +340,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars->s_free));
         const int kv0 = j * BN;
-        const bool diag = CAUSAL && (j == qt);
+        const bool diag = CAUSAL && (j == qt);  // key column e visible iff e <= r
         const bool tail = !CAUSAL && (kv0 + BN > p.N);
-        const int lim = diag ? (row - kv0) : (p.N - 1 - kv0);  // last allowed key column
+        const int lim = diag ? r : (p.N - 1 - kv0);  // last allowed key column
 #pragma unroll
         for (int e = 0; e < 128; ++e) {
           const float x = (diag || tail) && e > lim ? -INFINITY : __uint_as_float(s[e]);
@@ -367,9 +368,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
       for (int cc = 0; cc < HD / 32; ++cc) reg_fence32(a[cc]);
       if (valid) {
-        __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bh) * p.N + row) * HD;
+        __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bh) * p.N + row) * p.d;
 #pragma unroll
-        for (int cc = 0; cc < HD / 32; ++cc) store_row32_bf16(dst + cc * 32, a[cc], p.scale);
+        for (int cc = 0; cc < HD / 32; ++cc)
+          if (cc * 32 < p.d) store_row32_bf16(dst + cc * 32, a[cc], p.scale);
       }
     }
   }
@@ -596,14 +598,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     if (ok) {
       tc_fence_after();
       const bool valid = key < p.N;
-      const size_t off = (static_cast<size_t>(bh) * p.N + key) * HD;
+      const size_t off = (static_cast<size_t>(bh) * p.N + key) * p.d;
 #pragma unroll
       for (int cc = 0; cc < HD / 32; ++cc) {
         uint32_t a[32];
         tmem_ld32(lane_addr + BK_DV + cc * 32, a);
         tmem_wait_ld();
         reg_fence32(a);
-        if (valid) store_row32_bf16(p.dv + off + cc * 32, a, 1.f);
+        if (valid && cc * 32 < p.d) store_row32_bf16(p.dv + off + cc * 32, a, 1.f);
       }
 #pragma unroll
       for (int cc = 0; cc < HD / 32; ++cc) {
@@ -611,7 +613,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         tmem_ld32(lane_addr + BK_DK + cc * 32, a);
         tmem_wait_ld();
         reg_fence32(a);
-        if (valid) store_row32_bf16(p.dk + off + cc * 32, a, p.scale);
+        if (valid && cc * 32 < p.d) store_row32_bf16(p.dk + off + cc * 32, a, p.scale);
       }
     }
   }

@@ -677,6 +677,12 @@ static bool overlap(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
+// Head dimensions served: 64 and 128 natively; 32 and 96 by the 64- and
+// 128-column kernels, whose tiles TMA fills with zeros past d (loads) and
+// clips at d (stores), so the padding adds nothing to S, P V or the outputs.
+static bool d_supported(int d) { return d == 32 || d == 64 || d == 96 || d == 128; }
+static int padded_hd(int d) { return d <= 64 ? 64 : 128; }
+
 static int validate(const void* q, const void* k, const void* v, const void* o, const float* lse, int B, int H,
                     int N, int d, float scale) {
   if (!q || !k || !v || !o || !lse) {
@@ -692,8 +698,8 @@ static int validate(const void* q, const void* k, const void* v, const void* o, 
     set_detail("scale must be finite and positive");
     return FA2_ERR_INVALID_ARG;
   }
-  if (d != 64 && d != 128) {
-    set_detail("head dimension %d not supported (64 or 128)", d);
+  if (!d_supported(d)) {
+    set_detail("head dimension %d not supported (32, 64, 96 or 128)", d);
     return FA2_ERR_UNSUPPORTED;
   }
   const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
@@ -787,7 +793,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
   prm.timeout_ns = timeout_ns;
   prm.inject_timeout = inject;
-  if (d == 64)
+  if (padded_hd(d) == 64)
     return causal ? launch_t<64, true>(tq, tk, tv, to, prm, B, H, stream)
                   : launch_t<64, false>(tq, tk, tv, to, prm, B, H, stream);
   return causal ? launch_t<128, true>(tq, tk, tv, to, prm, B, H, stream)
@@ -863,7 +869,8 @@ static int skv_launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
   }
   if (prm.direct) return FA2_OK;
   const int rows = prm.BH * prm.Nq;
-  fa2_splitkv_combine_kernel<HD><<<(rows + 3) / 4, 128, 0, stream>>>(prm.o_part, prm.lse_part, o, lse, rows, splits);
+  fa2_splitkv_combine_kernel<HD><<<(rows + 3) / 4, 128, 0, stream>>>(prm.o_part, prm.lse_part, o, lse, rows, splits,
+                                                                      prm.d);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_detail("merge kernel launch: %s", cudaGetErrorString(e));
@@ -889,8 +896,8 @@ static int splitkv_impl(const void* q, const void* k, const void* v, void* o, fl
     set_detail("scale must be finite and positive");
     return FA2_ERR_INVALID_ARG;
   }
-  if (d != 64 && d != 128) {
-    set_detail("head dimension %d not supported (64 or 128)", d);
+  if (!d_supported(d)) {
+    set_detail("head dimension %d not supported (32, 64, 96 or 128)", d);
     return FA2_ERR_UNSUPPORTED;
   }
   const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
@@ -900,7 +907,7 @@ static int splitkv_impl(const void* q, const void* k, const void* v, void* o, fl
     return FA2_ERR_INVALID_ARG;
   }
   const int splits = skv_resolve_splits(B, H, Nq, Nk, n_splits);
-  const size_t need = skv_workspace_bytes(B, H, Nq, d, splits);
+  const size_t need = skv_workspace_bytes(B, H, Nq, padded_hd(d), splits);
   if (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)) {
     set_detail("workspace missing, misaligned or too small: %zu bytes, need %zu (256-byte aligned) for %d key ranges",
                workspace_bytes, need, splits);
@@ -928,9 +935,10 @@ static int splitkv_impl(const void* q, const void* k, const void* v, void* o, fl
   prm.o_part = prm.direct ? nullptr : static_cast<float*>(workspace);
   prm.lse_part = prm.direct ? nullptr
                             : reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                                       round256(static_cast<size_t>(splits) * BH * Nq * d * 4));
+                                                       round256(static_cast<size_t>(splits) * BH * Nq * padded_hd(d) * 4));
   prm.Nq = Nq;
   prm.Nk = Nk;
+  prm.d = d;
   prm.BH = static_cast<int>(BH);
   prm.n_kv_tiles = (Nk + BN - 1) / BN;
   prm.tiles_per_split = (prm.n_kv_tiles + splits - 1) / splits;
@@ -938,7 +946,7 @@ static int splitkv_impl(const void* q, const void* k, const void* v, void* o, fl
   prm.timeout_ns = DEFAULT_TIMEOUT_NS;
   const int n_q_tiles = (Nq + BM - 1) / BM;
   auto* ob = static_cast<__nv_bfloat16*>(o);
-  if (d == 64)
+  if (padded_hd(d) == 64)
     return causal ? skv_launch_t<64, true>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
                   : skv_launch_t<64, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
   return causal ? skv_launch_t<128, true>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
@@ -1008,8 +1016,8 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
     set_detail("scale must be finite and positive");
     return FA2_ERR_INVALID_ARG;
   }
-  if (d != 64 && d != 128) {
-    set_detail("head dimension %d not supported (64 or 128)", d);
+  if (!d_supported(d)) {
+    set_detail("head dimension %d not supported (32, 64, 96 or 128)", d);
     return FA2_ERR_UNSUPPORTED;
   }
   const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
@@ -1060,12 +1068,13 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   prm.dk = static_cast<__nv_bfloat16*>(dk);
   prm.dv = static_cast<__nv_bfloat16*>(dv);
   prm.N = N;
+  prm.d = d;
   prm.BH = static_cast<int>(BH);
   prm.group_heads = causal ? causal_group_heads(static_cast<int>(BH), N, d, prm.n_tiles) : 1;
   prm.scale = scale;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
   prm.timeout_ns = DEFAULT_TIMEOUT_NS;
-  if (d == 64)
+  if (padded_hd(d) == 64)
     return causal ? bwd_launch_t<64, true>(tq, tk, tv, tdo, prm, stream)
                   : bwd_launch_t<64, false>(tq, tk, tv, tdo, prm, stream);
   return causal ? bwd_launch_t<128, true>(tq, tk, tv, tdo, prm, stream)
@@ -1156,7 +1165,7 @@ int fa2_sync_status(void* stream) {
 }
 
 size_t fa2_fwd_host_workspace_bytes(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  if (B < 1 || H < 1 || N < 1 || !fa2::d_supported(d)) return 0;
   const size_t t = ((static_cast<size_t>(B) * H * N * d * 2) + 255) & ~static_cast<size_t>(255);
   const size_t l = ((static_cast<size_t>(B) * H * N * 4) + 255) & ~static_cast<size_t>(255);
   return 4 * t + l;
@@ -1171,7 +1180,7 @@ int fa2_fwd_host(const void* q, const void* k, const void* v, void* o, float* ls
   }
   const size_t need = fa2_fwd_host_workspace_bytes(B, H, N, d);
   if (need == 0) {
-    if (d != 64 && d != 128 && B >= 1 && H >= 1 && N >= 1) return FA2_ERR_UNSUPPORTED;
+    if (!fa2::d_supported(d) && B >= 1 && H >= 1 && N >= 1) return FA2_ERR_UNSUPPORTED;
     fa2::set_detail("bad sizes");
     return FA2_ERR_INVALID_ARG;
   }
@@ -1204,14 +1213,14 @@ int fa2_fwd_host(const void* q, const void* k, const void* v, void* o, float* ls
 }
 
 int fa2_fwd_splitkv_splits(int B, int H, int Nq, int Nk, int d, int n_splits) {
-  if (!fa2::skv_sizes_ok(B, H, Nq, Nk) || n_splits < 0 || (d != 64 && d != 128)) return 0;
+  if (!fa2::skv_sizes_ok(B, H, Nq, Nk) || n_splits < 0 || !fa2::d_supported(d)) return 0;
   return fa2::skv_resolve_splits(B, H, Nq, Nk, n_splits);
 }
 
 size_t fa2_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int n_splits) {
   const int splits = fa2_fwd_splitkv_splits(B, H, Nq, Nk, d, n_splits);
   if (splits == 0) return 0;
-  return fa2::skv_workspace_bytes(B, H, Nq, d, splits);
+  return fa2::skv_workspace_bytes(B, H, Nq, fa2::padded_hd(d), splits);
 }
 
 int fa2_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
@@ -1231,7 +1240,7 @@ int fa2_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o,
   size_t need = 0;
   if (fa2::skv_sizes_ok(B, H, Nq, Nk) && n_splits >= 0 && (d == 64 || d == 128)) {
     const int splits = fa2::skv_resolve_splits(B, H, Nq, Nk, n_splits);
-    need = fa2::skv_workspace_bytes(B, H, Nq, d, splits);
+    need = fa2::skv_workspace_bytes(B, H, Nq, fa2::padded_hd(d), splits);
     if (need > FA2_SPLITKV_STATIC_SCRATCH_BYTES) {
       fa2::set_detail("%d key ranges need %zu bytes of scratch; the static scratch holds %zu (fewer ranges need "
                       "less, one range none; fa2_fwd_splitkv takes a caller workspace of any size)",
@@ -1250,7 +1259,7 @@ int fa2_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o,
 }
 
 size_t fa2_bwd_workspace_bytes(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  if (B < 1 || H < 1 || N < 1 || !fa2::d_supported(d)) return 0;
   return fa2::bwd_workspace_bytes_for(B, H, N);
 }
 

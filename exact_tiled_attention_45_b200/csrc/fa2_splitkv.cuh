@@ -53,6 +53,7 @@ struct SkvParams {
   int direct;       // 1: one range, no merge step
   int Nq;
   int Nk;
+  int d;  // head dimension of q, k, v, o (<= HD; tiles are zero-padded to HD)
   int BH;
   int n_kv_tiles;       // ceil(Nk / 128)
   int tiles_per_split;  // key tiles per range
@@ -362,12 +363,12 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
         const float lse_row = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
         if (p.direct) {
           // One range: this is the final result (prow = bh * Nq + row).
-          uint4* dst = reinterpret_cast<uint4*>(p.o + prow * HD);
+          uint4* dst = reinterpret_cast<uint4*>(p.o + prow * p.d);
 #pragma unroll
           for (int c = 0; c < HD / 32; ++c)
 #pragma unroll
             for (int e = 0; e < 32; e += 8)
-              dst[c * 4 + e / 8] = make_uint4(
+              if (c * 32 < p.d) dst[c * 4 + e / 8] = make_uint4(
                   pack_bf16x2(__uint_as_float(o[c][e]) * inv_l, __uint_as_float(o[c][e + 1]) * inv_l),
                   pack_bf16x2(__uint_as_float(o[c][e + 2]) * inv_l, __uint_as_float(o[c][e + 3]) * inv_l),
                   pack_bf16x2(__uint_as_float(o[c][e + 4]) * inv_l, __uint_as_float(o[c][e + 5]) * inv_l),
@@ -402,7 +403,7 @@ template <int HD>
 __global__ void __launch_bounds__(128) fa2_splitkv_combine_kernel(const float* __restrict__ o_part,
                                                                   const float* __restrict__ lse_part,
                                                                   __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
-                                                                  int rows, int n_splits) {
+                                                                  int rows, int n_splits, int d) {
   const int row = static_cast<int>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -434,8 +435,10 @@ __global__ void __launch_bounds__(128) fa2_splitkv_combine_kernel(const float* _
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  __nv_bfloat16* dst = o + static_cast<size_t>(row) * HD + lane * PER;
-  if constexpr (PER == 4) {
+  __nv_bfloat16* dst = o + static_cast<size_t>(row) * d + lane * PER;
+  if (lane * PER >= d) {
+    // columns of the zero padding up to HD: nothing to store
+  } else if constexpr (PER == 4) {
     *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv),
                                                 pack_bf16x2(acc[2] * inv, acc[3] * inv));
   } else {

@@ -67,8 +67,9 @@ def _call(lib, q=FAKE, k=FAKE + (1 << 32), v=FAKE + (2 << 32), o=FAKE + (3 << 32
     (dict(B=70000), binding.FA2_ERR_INVALID_ARG),
     (dict(B=65535, H=65535), binding.FA2_ERR_INVALID_ARG),   # B*H >= 2^31
     (dict(B=1024, H=1024, N=2048 * 256), binding.FA2_ERR_INVALID_ARG),  # 2^31 CTAs
-    (dict(d=96), binding.FA2_ERR_UNSUPPORTED),
+    (dict(d=80), binding.FA2_ERR_UNSUPPORTED),
     (dict(d=256), binding.FA2_ERR_UNSUPPORTED),
+    (dict(d=16), binding.FA2_ERR_UNSUPPORTED),
     (dict(q=FAKE + 8), binding.FA2_ERR_INVALID_ARG),
     (dict(lse=FAKE + (4 << 32) + 2), binding.FA2_ERR_INVALID_ARG),
     (dict(o=FAKE), binding.FA2_ERR_INVALID_ARG),                   # o aliases q
@@ -144,7 +145,7 @@ def test_splitkv_split_count_and_workspace(lib):
     rows = s * 2 * 3 * 5
     r256 = lambda x: (x + 255) // 256 * 256
     assert lib.fa2_fwd_splitkv_workspace_bytes(2, 3, 5, 1000, 64, 3) == r256(rows * 64 * 4) + r256(rows * 4)
-    for bad in ((1, 1, 0, 10, 64, 0), (1, 1, 11, 10, 64, 0), (1, 1, 1, 10, 96, 0), (1, 1, 1, 10, 64, -1),
+    for bad in ((1, 1, 0, 10, 64, 0), (1, 1, 11, 10, 64, 0), (1, 1, 1, 10, 80, 0), (1, 1, 1, 10, 64, -1),
                 (300, 300, 1, 10, 64, 0)):
         assert lib.fa2_fwd_splitkv_workspace_bytes(*bad) == 0
         assert lib.fa2_fwd_splitkv_splits(*bad) == 0
@@ -174,7 +175,7 @@ def test_splitkv_auto_split_choice(lib):
     (dict(n_splits=-1), binding.FA2_ERR_INVALID_ARG),
     (dict(scale=0.0), binding.FA2_ERR_INVALID_ARG),
     (dict(scale=float("nan")), binding.FA2_ERR_INVALID_ARG),
-    (dict(d=96), binding.FA2_ERR_UNSUPPORTED),
+    (dict(d=80), binding.FA2_ERR_UNSUPPORTED),
     (dict(ws=FAKE + (5 << 32) + 128), binding.FA2_ERR_INVALID_ARG),  # workspace not 256-aligned
     (dict(ws_bytes=1024), binding.FA2_ERR_INVALID_ARG),              # workspace too small
     (dict(o=FAKE + (1 << 32)), binding.FA2_ERR_INVALID_ARG),         # o aliases k
@@ -217,7 +218,8 @@ def test_bwd_workspace_size(lib):
     assert lib.fa2_bwd_workspace_bytes(2, 3, 200, 128) == 2 * (2 * 3 * 256 * 4)
     assert lib.fa2_bwd_workspace_bytes(1, 1, 1, 64) == 2 * 512
     assert lib.fa2_bwd_workspace_bytes(1, 1, 0, 64) == 0
-    assert lib.fa2_bwd_workspace_bytes(1, 1, 8, 96) == 0
+    assert lib.fa2_bwd_workspace_bytes(1, 1, 8, 80) == 0
+    assert lib.fa2_bwd_workspace_bytes(1, 1, 8, 96) == 2 * 512  # d = 96 runs on zero-padded 128-column tiles
 
 
 @pytest.mark.parametrize("kw,expect", [
@@ -225,7 +227,7 @@ def test_bwd_workspace_size(lib):
     (dict(dv=0), binding.FA2_ERR_INVALID_ARG),
     (dict(ws=0), binding.FA2_ERR_INVALID_ARG),
     (dict(N=0), binding.FA2_ERR_INVALID_ARG),
-    (dict(d=96), binding.FA2_ERR_UNSUPPORTED),
+    (dict(d=80), binding.FA2_ERR_UNSUPPORTED),
     (dict(scale=0.0), binding.FA2_ERR_INVALID_ARG),
     (dict(scale=float("inf")), binding.FA2_ERR_INVALID_ARG),
     (dict(ws=FAKE + (9 << 32) + 64), binding.FA2_ERR_INVALID_ARG),   # workspace not 256-aligned
@@ -238,3 +240,13 @@ def test_bwd_workspace_size(lib):
 def test_bwd_bad_arguments_rejected_before_launch(lib, kw, expect):
     assert _bwd(lib, **kw) == expect
     assert lib.fa2_last_error_detail()
+
+
+def test_padded_head_dims_size_like_the_wider_kernel(lib):
+    # d = 32 and 96 run on the 64- and 128-column kernels; the split-K/V
+    # partials are kept at the padded width, the user tensors at d.
+    assert lib.fa2_fwd_splitkv_workspace_bytes(1, 2, 3, 1000, 96, 2) == lib.fa2_fwd_splitkv_workspace_bytes(
+        1, 2, 3, 1000, 128, 2)
+    assert lib.fa2_fwd_splitkv_workspace_bytes(1, 2, 3, 1000, 32, 2) == lib.fa2_fwd_splitkv_workspace_bytes(
+        1, 2, 3, 1000, 64, 2)
+    assert lib.fa2_fwd_host_workspace_bytes(1, 2, 128, 96) == 4 * (2 * 128 * 96 * 2) + 1024

@@ -67,6 +67,11 @@ CASES = [
     # large logits
     (1, 2, 512, 128, True, 4.0),
     (1, 2, 384, 64, False, 4.0),
+    # zero-padded head dims
+    (1, 2, 256, 32, False, 1.0),
+    (1, 2, 130, 32, True, 1.0),
+    (1, 2, 300, 96, True, 1.0),
+    (2, 1, 256, 96, False, 1.0),
 ]
 
 

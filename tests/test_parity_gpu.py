@@ -72,6 +72,13 @@ SMALL = [
     (2, 2, 512, 128, True, 4.0),
     (1, 2, 640, 64, False, 4.0),
     (1, 2, 640, 64, True, 4.0),
+    # head dims served by the zero-padded 64- and 128-column kernels
+    (1, 2, 256, 32, False, 1.0),
+    (1, 2, 256, 32, True, 1.0),
+    (2, 1, 129, 32, True, 4.0),
+    (1, 2, 300, 96, False, 1.0),
+    (2, 1, 333, 96, True, 1.0),
+    (1, 1, 1000, 96, False, 4.0),
 ]
 
 

@@ -64,6 +64,11 @@ CASES = [
     (2, 2, 1, 3000, 128, False, 0, 4.0),     # large logits
     (2, 2, 64, 3000, 128, True, 6, 4.0),
     (2, 2, 64, 3000, 64, True, 0, 4.0),
+    # zero-padded head dims
+    (1, 2, 1, 3000, 96, True, 0, 1.0),
+    (1, 2, 7, 2000, 32, False, 3, 1.0),
+    (1, 2, 130, 1500, 96, True, 5, 1.0),
+    (2, 1, 1, 900, 32, True, 1, 1.0),
 ]
 
 
