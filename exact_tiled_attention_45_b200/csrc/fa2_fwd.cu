@@ -236,14 +236,17 @@ __device__ __forceinline__ void softmax_role(const Params& p, const CUtensorMap*
       for (int e = 0; e < 128; ++e)
         if (e > lim) s[e] = __float_as_uint(-INFINITY);
     }
-    // Row max: eight independent 3-input chains, then combine.
+    // Row max: eight independent chains (3-input max over columns 8..119,
+    // then columns 120..127), then combine.
     float mx8[8];
 #pragma unroll
     for (int a = 0; a < 8; ++a) mx8[a] = __uint_as_float(s[a]);
 #pragma unroll
-    for (int e = 8; e < 128; e += 16)
+    for (int e = 8; e + 16 <= 128; e += 16)
 #pragma unroll
       for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], __uint_as_float(s[e + a]), __uint_as_float(s[e + 8 + a]));
+#pragma unroll
+    for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(mx8[a], __uint_as_float(s[120 + a]));
     const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
     const float m_cand = mx * c_log2;
     float m_new = m;
@@ -652,7 +655,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 // View a [B*H, N, d] bf16 tensor as a 3-D TMA map with 64 x 128 x 1 boxes,
 // 128-byte swizzle.  Rows past N read as zero.
-static int make_tmap(CUtensorMap* tm, const void* ptr, int d, int N, int BH) {
+static int make_tmap(CUtensorMap* tm, const void* ptr, int d, int N, int BH, int box_rows = 128) {
   auto enc = get_encode_fn();
   if (!enc) {
     set_detail("cuTensorMapEncodeTiled entry point unavailable");
@@ -660,7 +663,7 @@ static int make_tmap(CUtensorMap* tm, const void* ptr, int d, int N, int BH) {
   }
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -680,8 +683,10 @@ static bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 // Head dimensions served: 64 and 128 natively; 32 and 96 by the 64- and
 // 128-column kernels, whose tiles TMA fills with zeros past d (loads) and
 // clips at d (stores), so the padding adds nothing to S, P V or the outputs.
-static bool d_supported(int d) { return d == 32 || d == 64 || d == 96 || d == 128; }
-static int padded_hd(int d) { return d <= 64 ? 64 : 128; }
+static bool d_supported(int d) { return d == 32 || d == 64 || d == 96 || d == 128 || d == 256; }
+static int padded_hd(int d) { return d <= 64 ? 64 : (d <= 128 ? 128 : 256); }
+// Keys per tile of the split-K/V kernel: 64 at d = 256, else 128.
+static int skv_tile_keys(int d) { return padded_hd(d) == 256 ? 64 : 128; }
 
 static int validate(const void* q, const void* k, const void* v, const void* o, const float* lse, int B, int H,
                     int N, int d, float scale) {
@@ -699,7 +704,7 @@ static int validate(const void* q, const void* k, const void* v, const void* o, 
     return FA2_ERR_INVALID_ARG;
   }
   if (!d_supported(d)) {
-    set_detail("head dimension %d not supported (32, 64, 96 or 128)", d);
+    set_detail("head dimension %d not supported (32, 64, 96, 128 or 256)", d);
     return FA2_ERR_UNSUPPORTED;
   }
   const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
@@ -771,11 +776,24 @@ static int causal_group_heads(int BH, int N, int d, int n_q_blocks) {
   return (BH + groups - 1) / groups;
 }
 
+static int splitkv_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                        int Nk, int d, int causal, float scale, int n_splits, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream);
+
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                     int causal, float scale, unsigned long long timeout_ns, int inject, cudaStream_t stream) {
   g_detail[0] = 0;
   int st = validate(q, k, v, o, lse, B, H, N, d, scale);
   if (st != FA2_OK) return st;
+  if (padded_hd(d) == 256) {
+    // d = 256 runs on the one-tile kernel of the split-K/V path (64-key tiles)
+    // as a single key range with Nq = Nk, which writes O and LSE directly.
+    if (inject) {
+      set_detail("the timeout test hook covers the 32..128-column kernel only");
+      return FA2_ERR_UNSUPPORTED;
+    }
+    return splitkv_impl(q, k, v, o, lse, B, H, N, N, d, causal, scale, 1, nullptr, 0, stream);
+  }
   CUtensorMap tq, tk, tv, to;
   const int BH = B * H;
   if ((st = make_tmap(&tq, q, d, N, BH)) != FA2_OK) return st;
@@ -817,8 +835,8 @@ static bool skv_sizes_ok(int B, int H, int Nq, int Nk) {
 // keeping at least 4 key tiles per range.  A requested count is capped at 128
 // and at the number of key tiles, then reduced to ceil(tiles / ceil(tiles /
 // s)) so that no range is empty by construction.
-static int skv_resolve_splits(int B, int H, int Nq, int Nk, int n_splits) {
-  const int n_kv = (Nk + BN - 1) / BN;
+static int skv_resolve_splits(int B, int H, int Nq, int Nk, int n_splits, int tile_keys) {
+  const int n_kv = (Nk + tile_keys - 1) / tile_keys;
   int s = n_splits;
   if (s <= 0) {
     const long long base = static_cast<long long>((Nq + BM - 1) / BM) * B * H;
@@ -897,7 +915,7 @@ static int splitkv_impl(const void* q, const void* k, const void* v, void* o, fl
     return FA2_ERR_INVALID_ARG;
   }
   if (!d_supported(d)) {
-    set_detail("head dimension %d not supported (32, 64, 96 or 128)", d);
+    set_detail("head dimension %d not supported (32, 64, 96, 128 or 256)", d);
     return FA2_ERR_UNSUPPORTED;
   }
   const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
@@ -906,7 +924,7 @@ static int splitkv_impl(const void* q, const void* k, const void* v, void* o, fl
     set_detail("misaligned pointer (q/k/v/o need 16 bytes, lse 4)");
     return FA2_ERR_INVALID_ARG;
   }
-  const int splits = skv_resolve_splits(B, H, Nq, Nk, n_splits);
+  const int splits = skv_resolve_splits(B, H, Nq, Nk, n_splits, skv_tile_keys(d));
   const size_t need = skv_workspace_bytes(B, H, Nq, padded_hd(d), splits);
   if (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)) {
     set_detail("workspace missing, misaligned or too small: %zu bytes, need %zu (256-byte aligned) for %d key ranges",
@@ -926,8 +944,8 @@ static int splitkv_impl(const void* q, const void* k, const void* v, void* o, fl
   CUtensorMap tq, tk, tv;
   int st;
   if ((st = make_tmap(&tq, q, d, Nq, static_cast<int>(BH))) != FA2_OK) return st;
-  if ((st = make_tmap(&tk, k, d, Nk, static_cast<int>(BH))) != FA2_OK) return st;
-  if ((st = make_tmap(&tv, v, d, Nk, static_cast<int>(BH))) != FA2_OK) return st;
+  if ((st = make_tmap(&tk, k, d, Nk, static_cast<int>(BH), skv_tile_keys(d))) != FA2_OK) return st;
+  if ((st = make_tmap(&tv, v, d, Nk, static_cast<int>(BH), skv_tile_keys(d))) != FA2_OK) return st;
   SkvParams prm;
   prm.direct = splits == 1;
   prm.o = static_cast<__nv_bfloat16*>(o);
@@ -940,7 +958,7 @@ static int splitkv_impl(const void* q, const void* k, const void* v, void* o, fl
   prm.Nk = Nk;
   prm.d = d;
   prm.BH = static_cast<int>(BH);
-  prm.n_kv_tiles = (Nk + BN - 1) / BN;
+  prm.n_kv_tiles = (Nk + skv_tile_keys(d) - 1) / skv_tile_keys(d);
   prm.tiles_per_split = (prm.n_kv_tiles + splits - 1) / splits;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
   prm.timeout_ns = DEFAULT_TIMEOUT_NS;
@@ -949,6 +967,9 @@ static int splitkv_impl(const void* q, const void* k, const void* v, void* o, fl
   if (padded_hd(d) == 64)
     return causal ? skv_launch_t<64, true>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
                   : skv_launch_t<64, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
+  if (padded_hd(d) == 256)
+    return causal ? skv_launch_t<256, true>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
+                  : skv_launch_t<256, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
   return causal ? skv_launch_t<128, true>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
                 : skv_launch_t<128, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
 }
@@ -1016,8 +1037,8 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
     set_detail("scale must be finite and positive");
     return FA2_ERR_INVALID_ARG;
   }
-  if (!d_supported(d)) {
-    set_detail("head dimension %d not supported (32, 64, 96 or 128)", d);
+  if (!d_supported(d) || padded_hd(d) == 256) {
+    set_detail("head dimension %d not supported by the backward (32, 64, 96 or 128)", d);
     return FA2_ERR_UNSUPPORTED;
   }
   const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
@@ -1214,7 +1235,7 @@ int fa2_fwd_host(const void* q, const void* k, const void* v, void* o, float* ls
 
 int fa2_fwd_splitkv_splits(int B, int H, int Nq, int Nk, int d, int n_splits) {
   if (!fa2::skv_sizes_ok(B, H, Nq, Nk) || n_splits < 0 || !fa2::d_supported(d)) return 0;
-  return fa2::skv_resolve_splits(B, H, Nq, Nk, n_splits);
+  return fa2::skv_resolve_splits(B, H, Nq, Nk, n_splits, fa2::skv_tile_keys(d));
 }
 
 size_t fa2_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int n_splits) {
@@ -1239,7 +1260,7 @@ int fa2_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o,
   }
   size_t need = 0;
   if (fa2::skv_sizes_ok(B, H, Nq, Nk) && n_splits >= 0 && (d == 64 || d == 128)) {
-    const int splits = fa2::skv_resolve_splits(B, H, Nq, Nk, n_splits);
+    const int splits = fa2::skv_resolve_splits(B, H, Nq, Nk, n_splits, fa2::skv_tile_keys(d));
     need = fa2::skv_workspace_bytes(B, H, Nq, fa2::padded_hd(d), splits);
     if (need > FA2_SPLITKV_STATIC_SCRATCH_BYTES) {
       fa2::set_detail("%d key ranges need %zu bytes of scratch; the static scratch holds %zu (fewer ranges need "
@@ -1259,7 +1280,7 @@ int fa2_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o,
 }
 
 size_t fa2_bwd_workspace_bytes(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || !fa2::d_supported(d)) return 0;
+  if (B < 1 || H < 1 || N < 1 || !fa2::d_supported(d) || fa2::padded_hd(d) == 256) return 0;
   return fa2::bwd_workspace_bytes_for(B, H, N);
 }
 

@@ -22,27 +22,38 @@
 // TMA producer, warp 5 MMA issuer.  TMEM: two score buffers (the next S is
 // computed while the softmax works on the current one), a separate P buffer,
 // and O.  Rows past Nq are computed on zero queries and never stored.
+//
+// Head dimension 256 (also served to the square entry point as one range with
+// Nq = Nk): 64-key tiles, so that a 256-column O accumulator, two score
+// buffers and P fit the 512 TMEM columns and two stages of K and V fit shared
+// memory next to the 64 KB query tile.
 
 constexpr int SKV_THREADS = 192;
 constexpr int SKV_PRODUCER_WARP = 4;
 constexpr int SKV_MMA_WARP = 5;
-constexpr uint32_t SKV_TM_S0 = 0, SKV_TM_S1 = 128, SKV_TM_P = 256, SKV_TM_O = 384;
 
 template <int HD>
 struct SkvCfg {
-  static constexpr int KCH = HD / 64;
-  static constexpr int CHUNK_BYTES = 128 * 128;
-  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;
-  // Deep K/V rings: the stream over keys is the bound, so keep many tiles in
-  // flight (224 KB of rings for d = 128, 128 KB for d = 64).
-  static constexpr int KS = (HD == 128) ? 3 : 4;
+  static constexpr int SBN = (HD == 256) ? 64 : 128;  // keys per tile
+  static constexpr int KCH = HD / 64;                 // 64-column (128-byte) chunks
+  static constexpr int Q_CHUNK = 128 * 128;           // 128 query rows x 128 bytes
+  static constexpr int KV_CHUNK = SBN * 128;          // SBN key rows x 128 bytes
+  static constexpr int Q_BYTES = KCH * Q_CHUNK;
+  static constexpr int KV_BYTES = KCH * KV_CHUNK;
+  // Deep K/V rings: the stream over keys is the bound for few queries, so
+  // keep many tiles in flight (224 KB of rings for d = 128, 128 KB for d = 64,
+  // 128 KB for d = 256).
+  static constexpr int KS = (HD == 64) ? 4 : (HD == 128 ? 3 : 2);
   static constexpr int VS = KS;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + TILE_BYTES;
-  static constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_V + VS * TILE_BYTES;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + KS * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VS * KV_BYTES;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  // TMEM columns: S0, S1 (SBN each), P (SBN/2 packed bf16 pairs), O (HD).
+  static constexpr uint32_t TM_S0 = 0, TM_S1 = SBN, TM_P = 2 * SBN, TM_O = (HD == 256) ? 256 : 384;
+  static_assert(TM_P + SBN / 2 <= TM_O && TM_O + HD <= 512, "TMEM budget");
 };
 
 struct SkvParams {
@@ -55,7 +66,7 @@ struct SkvParams {
   int Nk;
   int d;  // head dimension of q, k, v, o (<= HD; tiles are zero-padded to HD)
   int BH;
-  int n_kv_tiles;       // ceil(Nk / 128)
+  int n_kv_tiles;       // ceil(Nk / SBN)
   int tiles_per_split;  // key tiles per range
   float scale_log2;
   unsigned long long timeout_ns;
@@ -86,7 +97,7 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
   // Key tiles this query tile needs: all of them, or (causal) up to the
   // position of its last row.
   int n_need = p.n_kv_tiles;
-  if (CAUSAL) n_need = min(n_need, (offset + min(q_first + BM, p.Nq) - 1) / BN + 1);
+  if (CAUSAL) n_need = min(n_need, (offset + min(q_first + BM, p.Nq) - 1) / C::SBN + 1);
   const int kt_begin = split * p.tiles_per_split;
   const int kt_end = min(kt_begin + p.tiles_per_split, n_need);
   const int nkv = kt_end - kt_begin;
@@ -160,28 +171,28 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
   if (warp == SKV_PRODUCER_WARP) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(b_q, C::TILE_BYTES);
-      for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * C::CHUNK_BYTES, &tm_q, b_q, c * 64, q_first, bh);
+      mbar_arrive_expect_tx(b_q, C::Q_BYTES);
+      for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * C::Q_CHUNK, &tm_q, b_q, c * 64, q_first, bh);
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < nkv; ++j) {
-        const int kv0 = (kt_begin + j) * BN;
+        const int kv0 = (kt_begin + j) * C::SBN;
         const int ks = j % C::KS;
         if (j >= C::KS &&
             !wait_bounded(smem_u32(&bars->k_empty[ks]), ((j / C::KS) - 1) & 1, abort_flag, to, ROLE_PRODUCER))
           break;
         const uint32_t kb = smem_u32(&bars->k_full[ks]);
-        mbar_arrive_expect_tx(kb, C::TILE_BYTES);
+        mbar_arrive_expect_tx(kb, C::KV_BYTES);
         for (int c = 0; c < C::KCH; ++c)
-          tma_load_3d(sK + ks * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_k, kb, c * 64, kv0, bh);
+          tma_load_3d(sK + ks * C::KV_BYTES + c * C::KV_CHUNK, &tm_k, kb, c * 64, kv0, bh);
         ++k_issued;
         const int vs = j % C::VS;
         if (j >= C::VS &&
             !wait_bounded(smem_u32(&bars->v_empty[vs]), ((j / C::VS) - 1) & 1, abort_flag, to, ROLE_PRODUCER))
           break;
         const uint32_t vb = smem_u32(&bars->v_full[vs]);
-        mbar_arrive_expect_tx(vb, C::TILE_BYTES);
+        mbar_arrive_expect_tx(vb, C::KV_BYTES);
         for (int c = 0; c < C::KCH; ++c)
-          tma_load_3d(sV + vs * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_v, vb, c * 64, kv0, bh);
+          tma_load_3d(sV + vs * C::KV_BYTES + c * C::KV_CHUNK, &tm_v, vb, c * 64, kv0, bh);
         ++v_issued;
       }
       wait_drain(b_q, 0, to);
@@ -195,7 +206,7 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
     // Order S(0), S(1), PV(0), S(2), PV(1), ...: the next scores are computed
     // while the softmax works on the current ones.
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, C::SBN, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
       bool ok = wait_bounded(b_q, 0, abort_flag, to, ROLE_MMA);
       for (int j = 0; ok && j <= nkv; ++j) {
@@ -206,13 +217,13 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
           if (j >= 2 && !wait_bounded(smem_u32(&bars->s_free[sb]), ((j - 2) >> 1) & 1, abort_flag, to, ROLE_MMA))
             break;
           tc_fence_after();
-          const uint32_t d_s = tmem + (sb ? SKV_TM_S1 : SKV_TM_S0);
-          const uint32_t kbase = sK + ks * C::TILE_BYTES;
+          const uint32_t d_s = tmem + (sb ? C::TM_S1 : C::TM_S0);
+          const uint32_t kbase = sK + ks * C::KV_BYTES;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-            mma_ss(d_s, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024), IDESC_S,
-                   kk > 0 ? 1u : 0u);
+            const uint32_t in_chunk = (kk & 3) * 32;
+            mma_ss(d_s, smem_desc_sw128(sQ + (kk >> 2) * C::Q_CHUNK + in_chunk, 16, 1024),
+                   smem_desc_sw128(kbase + (kk >> 2) * C::KV_CHUNK + in_chunk, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
           }
           mma_commit(smem_u32(&bars->s_full[sb]));
           mma_commit(smem_u32(&bars->k_empty[ks]));
@@ -223,11 +234,11 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
           if (!wait_bounded(b_p, i & 1, abort_flag, to, ROLE_MMA)) break;
           if (!wait_bounded(smem_u32(&bars->v_full[vs]), (i / C::VS) & 1, abort_flag, to, ROLE_MMA)) break;
           tc_fence_after();
-          const uint32_t vbase = sV + vs * C::TILE_BYTES;
+          const uint32_t vbase = sV + vs * C::KV_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            mma_ts(tmem + SKV_TM_O, tmem + SKV_TM_P + kk * 8,
-                   smem_desc_sw128(vbase + kk * 2048, C::CHUNK_BYTES, 1024), IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < C::SBN / 16; ++kk)
+            mma_ts(tmem + C::TM_O, tmem + C::TM_P + kk * 8,
+                   smem_desc_sw128(vbase + kk * 2048, C::KV_CHUNK, 1024), IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
           mma_commit(smem_u32(&bars->v_empty[vs]));
           mma_commit(b_pv);
         }
@@ -253,36 +264,40 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
       ok = wait_warp(smem_u32(&bars->s_full[sb]), (i >> 1) & 1, abort_flag, to);
       if (!ok) break;
       tc_fence_after();
-      const int kv0 = (kt_begin + i) * BN;
-      uint32_t pk[2][32];
+      constexpr int SBN = C::SBN;
+      const int kv0 = (kt_begin + i) * SBN;
+      uint32_t pk[SBN / 64][32];
       float alpha = 1.f, rowsum = 0.f, m_new = m;
       bool rescale = false;
       if (live) {
-        uint32_t s[128];
-        const uint32_t s_addr = lane_addr + (sb ? SKV_TM_S1 : SKV_TM_S0);
+        uint32_t s[SBN];
+        const uint32_t s_addr = lane_addr + (sb ? C::TM_S1 : C::TM_S0);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
+        for (int c = 0; c < SBN / 32; ++c)
+          tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
+        for (int c = 0; c < SBN / 32; ++c) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[sb]));
         // Mask: keys past the row's position (causal) or past Nk.
         const int lim = CAUSAL ? min(pos, p.Nk - 1) - kv0 : p.Nk - 1 - kv0;
-        if (lim < BN - 1) {
+        if (lim < SBN - 1) {
 #pragma unroll
-          for (int e = 0; e < 128; ++e)
+          for (int e = 0; e < SBN; ++e)
             if (e > lim) s[e] = __float_as_uint(-INFINITY);
         }
         float mx8[8];
 #pragma unroll
         for (int a = 0; a < 8; ++a) mx8[a] = __uint_as_float(s[a]);
 #pragma unroll
-        for (int e = 8; e < 128; e += 16)
+        for (int e = 8; e + 16 <= SBN; e += 16)  // columns 8 .. SBN-9
 #pragma unroll
           for (int a = 0; a < 8; ++a)
             mx8[a] = fmax3(mx8[a], __uint_as_float(s[e + a]), __uint_as_float(s[e + 8 + a]));
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(mx8[a], __uint_as_float(s[SBN - 8 + a]));  // the last 8
         const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         const float m_cand = mx * c_log2;
         if (m_cand > m + RESCALE_THRESHOLD) m_new = m_cand;
@@ -292,7 +307,7 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
         const uint64_t mm = f2_pack(-m_use, -m_use);
         uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < SBN / 32; ++c) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const uint64_t x =
@@ -323,7 +338,7 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < HD / 32; ++c) {
             uint32_t o[32];
-            tmem_ld32(lane_addr + SKV_TM_O + c * 32, o);
+            tmem_ld32(lane_addr + C::TM_O + c * 32, o);
             tmem_wait_ld();
             reg_fence32(o);
 #pragma unroll
@@ -333,13 +348,13 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
               o[e] = __float_as_uint(a0);
               o[e + 1] = __float_as_uint(a1);
             }
-            tmem_st32(lane_addr + SKV_TM_O + c * 32, o);
+            tmem_st32(lane_addr + C::TM_O + c * 32, o);
           }
         }
       }
       if (live) {
-        tmem_st32(lane_addr + SKV_TM_P, pk[0]);
-        tmem_st32(lane_addr + SKV_TM_P + 32, pk[1]);
+#pragma unroll
+        for (int h = 0; h < SBN / 64; ++h) tmem_st32(lane_addr + C::TM_P + 32 * h, pk[h]);
         tmem_wait_st();
       }
       tc_fence_before();
@@ -351,40 +366,42 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
     if (ok) ok = wait_warp(b_pv, (nkv - 1) & 1, abort_flag, to);
     if (ok && live) {
       tc_fence_after();
-      uint32_t o[HD / 32][32];
+      const bool store = row < p.Nq;
+      const size_t prow = (static_cast<size_t>(split) * p.BH + bh) * p.Nq + row;
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      // 32 columns at a time (a 256-column O does not fit in registers).
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) tmem_ld32(lane_addr + SKV_TM_O + c * 32, o[c]);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < HD / 32; ++c) reg_fence32(o[c]);
-      if (row < p.Nq) {
-        const size_t prow = (static_cast<size_t>(split) * p.BH + bh) * p.Nq + row;
-        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-        const float lse_row = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(lane_addr + C::TM_O + c * 32, o);
+        tmem_wait_ld();
+        reg_fence32(o);
+        if (!store) continue;
         if (p.direct) {
           // One range: this is the final result (prow = bh * Nq + row).
-          uint4* dst = reinterpret_cast<uint4*>(p.o + prow * p.d);
-#pragma unroll
-          for (int c = 0; c < HD / 32; ++c)
+          if (c * 32 < p.d) {
+            uint4* dst = reinterpret_cast<uint4*>(p.o + prow * p.d + c * 32);
 #pragma unroll
             for (int e = 0; e < 32; e += 8)
-              if (c * 32 < p.d) dst[c * 4 + e / 8] = make_uint4(
-                  pack_bf16x2(__uint_as_float(o[c][e]) * inv_l, __uint_as_float(o[c][e + 1]) * inv_l),
-                  pack_bf16x2(__uint_as_float(o[c][e + 2]) * inv_l, __uint_as_float(o[c][e + 3]) * inv_l),
-                  pack_bf16x2(__uint_as_float(o[c][e + 4]) * inv_l, __uint_as_float(o[c][e + 5]) * inv_l),
-                  pack_bf16x2(__uint_as_float(o[c][e + 6]) * inv_l, __uint_as_float(o[c][e + 7]) * inv_l));
-          p.lse[prow] = lse_row;
+              dst[e / 8] = make_uint4(pack_bf16x2(__uint_as_float(o[e]) * inv_l, __uint_as_float(o[e + 1]) * inv_l),
+                                      pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l),
+                                      pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l),
+                                      pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l));
+          }
         } else {
-          float4* dst = reinterpret_cast<float4*>(p.o_part + prow * HD);
+          float4* dst = reinterpret_cast<float4*>(p.o_part + prow * HD + c * 32);
 #pragma unroll
-          for (int c = 0; c < HD / 32; ++c)
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              dst[c * 8 + e / 4] =
-                  make_float4(__uint_as_float(o[c][e]) * inv_l, __uint_as_float(o[c][e + 1]) * inv_l,
-                              __uint_as_float(o[c][e + 2]) * inv_l, __uint_as_float(o[c][e + 3]) * inv_l);
-          p.lse_part[prow] = lse_row;
+          for (int e = 0; e < 32; e += 4)
+            dst[e / 4] = make_float4(__uint_as_float(o[e]) * inv_l, __uint_as_float(o[e + 1]) * inv_l,
+                                     __uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
         }
+      }
+      if (store) {
+        const float lse_row = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (p.direct)
+          p.lse[prow] = lse_row;
+        else
+          p.lse_part[prow] = lse_row;
       }
     }
   }
@@ -407,7 +424,7 @@ __global__ void __launch_bounds__(128) fa2_splitkv_combine_kernel(const float* _
   const int row = static_cast<int>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
-  constexpr int PER = HD / 32;  // 4 (d = 128) or 2 (d = 64) columns per lane
+  constexpr int PER = HD / 32;  // 8 (d = 256), 4 (d = 128) or 2 (d = 64) columns per lane
   float mx = -INFINITY;
   for (int s = 0; s < n_splits; ++s) mx = fmaxf(mx, lse_part[static_cast<size_t>(s) * rows + row]);
   float acc[PER];
@@ -421,12 +438,15 @@ __global__ void __launch_bounds__(128) fa2_splitkv_combine_kernel(const float* _
       const float w = __expf(ls - mx);
       wsum += w;
       const float* src = o_part + (static_cast<size_t>(s) * rows + row) * HD + lane * PER;
-      if constexpr (PER == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(src);
-        acc[0] += w * x.x;
-        acc[1] += w * x.y;
-        acc[2] += w * x.z;
-        acc[3] += w * x.w;
+      if constexpr (PER >= 4) {
+#pragma unroll
+        for (int q4 = 0; q4 < PER / 4; ++q4) {
+          const float4 x = *reinterpret_cast<const float4*>(src + 4 * q4);
+          acc[4 * q4] += w * x.x;
+          acc[4 * q4 + 1] += w * x.y;
+          acc[4 * q4 + 2] += w * x.z;
+          acc[4 * q4 + 3] += w * x.w;
+        }
       } else {
         const float2 x = *reinterpret_cast<const float2*>(src);
         acc[0] += w * x.x;
@@ -438,6 +458,9 @@ __global__ void __launch_bounds__(128) fa2_splitkv_combine_kernel(const float* _
   __nv_bfloat16* dst = o + static_cast<size_t>(row) * d + lane * PER;
   if (lane * PER >= d) {
     // columns of the zero padding up to HD: nothing to store
+  } else if constexpr (PER == 8) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                                                pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
   } else if constexpr (PER == 4) {
     *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv),
                                                 pack_bf16x2(acc[2] * inv, acc[3] * inv));

@@ -100,7 +100,7 @@ class DecodeWorkload:
 
 def _grid():
     out = []
-    for d in (64, 128):
+    for d in (64, 128, 256):
         for causal in (False, True):
             for N in (512, 1024, 2048, 4096, 8192, 16384):
                 H = 2048 // d

@@ -42,7 +42,7 @@ extern "C" {
 typedef enum {
   FA2_OK = 0,
   FA2_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, aliasing, non-finite scale */
-  FA2_ERR_UNSUPPORTED = 2, /* valid request the library does not implement (e.g. d not in {32,64,96,128}) */
+  FA2_ERR_UNSUPPORTED = 2, /* valid request the library does not implement (e.g. d not in {32,64,96,128,256}) */
   FA2_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed; see fa2_last_error_detail() */
   FA2_ERR_TIMEOUT = 4      /* a kernel's bounded wait gave up (reported by fa2_sync_status) */
 } fa2_status;
@@ -57,9 +57,11 @@ typedef enum {
  *             written with the natural-log logsumexp of the scaled scores.
  *   B, H, N : >= 1; B <= 65535, H <= 65535, B*H < 2^31, N <= 16776960.
  *             Any such N works (a ragged last tile is masked).
- *   d       : head dimension, 32, 64, 96 or 128 (others -> FA2_ERR_UNSUPPORTED).
- *             32 and 96 run on the 64- and 128-column kernels with the
- *             extra columns zero-filled on load and clipped on store.
+ *   d       : head dimension, 32, 64, 96, 128 or 256 (others ->
+ *             FA2_ERR_UNSUPPORTED).  32 and 96 run on the 64- and 128-column
+ *             kernels with the extra columns zero-filled on load and clipped
+ *             on store; 256 runs on the one-query-tile kernel of
+ *             fa2_fwd_splitkv with 64-key tiles (a single key range).
  *   causal  : 0 = every key; non-zero = key j allowed only for query i >= j.
  *   scale   : multiplier of q.k, finite and > 0 (the usual choice is
  *             1/sqrt(d)); other values -> FA2_ERR_INVALID_ARG.
@@ -92,7 +94,7 @@ int fa2_sync_status(void* stream);
 
 /*
  * Test hook for the failure path: launch the attention kernel (same
- * arguments as fa2_fwd) with the query-tile load withheld, so every wait on it
+ * arguments as fa2_fwd, d <= 128) with the query-tile load withheld, so every wait on it
  * runs out after `timeout_ns` nanoseconds.  The kernel then sets the status
  * word and exits cleanly (tensor memory released, no copy left in flight);
  * fa2_sync_status returns FA2_ERR_TIMEOUT.  Outputs are unspecified.
@@ -120,7 +122,7 @@ int fa2_fwd_inject_timeout(const void* q, const void* k, const void* v, void* o,
  *   Nq, Nk  : 1 <= Nq <= Nk.  Query row i is sequence position Nk - Nq + i
  *             (the last Nq positions); with Nq == Nk this is fa2_fwd.
  *   B, H    : >= 1 with B*H <= 65535.
- *   d       : 32, 64, 96 or 128 (others -> FA2_ERR_UNSUPPORTED).
+ *   d       : 32, 64, 96, 128 or 256 (others -> FA2_ERR_UNSUPPORTED).
  *   causal  : 0 = every key; non-zero = key j allowed for query row i only if
  *             j <= Nk - Nq + i.
  *   scale   : finite and > 0.
@@ -171,7 +173,8 @@ size_t fa2_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int 
  *   lse     : device pointer, fp32 [B,H,N], natural log, 4-byte aligned.
  *   dq, dk, dv : device pointers, bf16 [B,H,N,d]; written.  They must not
  *             overlap each other, the inputs or the workspace.
- *   B, H, N, d, causal, scale : as for fa2_fwd (d 32, 64, 96 or 128; scale > 0).
+ *   B, H, N, d, causal, scale : as for fa2_fwd, but d 32, 64, 96 or 128
+ *             (256 -> FA2_ERR_UNSUPPORTED); scale > 0.
  *   workspace, workspace_bytes : caller-owned device buffer, 256-byte
  *             aligned, of at least fa2_bwd_workspace_bytes(B,H,N,d) bytes;
  *             it carries per-row LSE*log2(e) and rowsum(dO o O) from the

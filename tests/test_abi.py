@@ -68,7 +68,7 @@ def _call(lib, q=FAKE, k=FAKE + (1 << 32), v=FAKE + (2 << 32), o=FAKE + (3 << 32
     (dict(B=65535, H=65535), binding.FA2_ERR_INVALID_ARG),   # B*H >= 2^31
     (dict(B=1024, H=1024, N=2048 * 256), binding.FA2_ERR_INVALID_ARG),  # 2^31 CTAs
     (dict(d=80), binding.FA2_ERR_UNSUPPORTED),
-    (dict(d=256), binding.FA2_ERR_UNSUPPORTED),
+    (dict(d=512), binding.FA2_ERR_UNSUPPORTED),
     (dict(d=16), binding.FA2_ERR_UNSUPPORTED),
     (dict(q=FAKE + 8), binding.FA2_ERR_INVALID_ARG),
     (dict(lse=FAKE + (4 << 32) + 2), binding.FA2_ERR_INVALID_ARG),
@@ -219,6 +219,7 @@ def test_bwd_workspace_size(lib):
     assert lib.fa2_bwd_workspace_bytes(1, 1, 1, 64) == 2 * 512
     assert lib.fa2_bwd_workspace_bytes(1, 1, 0, 64) == 0
     assert lib.fa2_bwd_workspace_bytes(1, 1, 8, 80) == 0
+    assert lib.fa2_bwd_workspace_bytes(1, 1, 8, 256) == 0  # the backward serves d <= 128
     assert lib.fa2_bwd_workspace_bytes(1, 1, 8, 96) == 2 * 512  # d = 96 runs on zero-padded 128-column tiles
 
 
@@ -228,6 +229,7 @@ def test_bwd_workspace_size(lib):
     (dict(ws=0), binding.FA2_ERR_INVALID_ARG),
     (dict(N=0), binding.FA2_ERR_INVALID_ARG),
     (dict(d=80), binding.FA2_ERR_UNSUPPORTED),
+    (dict(d=256), binding.FA2_ERR_UNSUPPORTED),
     (dict(scale=0.0), binding.FA2_ERR_INVALID_ARG),
     (dict(scale=float("inf")), binding.FA2_ERR_INVALID_ARG),
     (dict(ws=FAKE + (9 << 32) + 64), binding.FA2_ERR_INVALID_ARG),   # workspace not 256-aligned
@@ -250,3 +252,13 @@ def test_padded_head_dims_size_like_the_wider_kernel(lib):
     assert lib.fa2_fwd_splitkv_workspace_bytes(1, 2, 3, 1000, 32, 2) == lib.fa2_fwd_splitkv_workspace_bytes(
         1, 2, 3, 1000, 64, 2)
     assert lib.fa2_fwd_host_workspace_bytes(1, 2, 128, 96) == 4 * (2 * 128 * 96 * 2) + 1024
+
+
+def test_head_dim_256_uses_64_key_tiles(lib):
+    # d = 256 runs on the one-tile kernel with 64-key tiles: 1000 keys are 16
+    # tiles (8 at 128 keys), so up to 16 ranges and >= 4 tiles per range.
+    assert lib.fa2_fwd_splitkv_splits(1, 1, 1, 1000, 256, 500) == 16
+    assert lib.fa2_fwd_splitkv_splits(1, 1, 1, 1000, 128, 500) == 8
+    assert lib.fa2_fwd_splitkv_splits(1, 1, 1, 1000, 256, 0) == 4
+    rows = 2 * 1 * 2 * 3
+    assert lib.fa2_fwd_splitkv_workspace_bytes(1, 2, 3, 1000, 256, 2) == (rows * 256 * 4 + 255) // 256 * 256 + 256

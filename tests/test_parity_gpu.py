@@ -79,6 +79,13 @@ SMALL = [
     (1, 2, 300, 96, False, 1.0),
     (2, 1, 333, 96, True, 1.0),
     (1, 1, 1000, 96, False, 4.0),
+    # d = 256: the one-tile kernel with 64-key tiles, one key range
+    (1, 2, 256, 256, False, 1.0),
+    (1, 2, 256, 256, True, 1.0),
+    (2, 1, 321, 256, True, 1.0),
+    (1, 1, 1, 256, False, 1.0),
+    (1, 2, 700, 256, False, 4.0),
+    (1, 2, 640, 256, True, 4.0),
 ]
 
 

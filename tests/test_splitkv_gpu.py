@@ -69,6 +69,11 @@ CASES = [
     (1, 2, 7, 2000, 32, False, 3, 1.0),
     (1, 2, 130, 1500, 96, True, 5, 1.0),
     (2, 1, 1, 900, 32, True, 1, 1.0),
+    # d = 256: 64-key tiles
+    (2, 2, 1, 4000, 256, True, 0, 1.0),
+    (1, 2, 3, 1500, 256, False, 7, 1.0),
+    (1, 2, 130, 1000, 256, True, 3, 4.0),
+    (1, 1, 1, 65, 256, False, 2, 1.0),
 ]
 
 
