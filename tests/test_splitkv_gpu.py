@@ -69,6 +69,12 @@ CASES = [
     (1, 2, 7, 2000, 32, False, 3, 1.0),
     (1, 2, 130, 1500, 96, True, 5, 1.0),
     (2, 1, 1, 900, 32, True, 1, 1.0),
+    # two to four queries, long and short key ranges
+    (1, 3, 2, 777, 128, True, 0, 1.0),
+    (2, 2, 4, 3001, 64, False, 3, 1.0),
+    (1, 2, 4, 4, 256, True, 0, 1.0),
+    (2, 1, 3, 33, 128, True, 2, 4.0),
+    (1, 2, 1, 20000, 64, True, 0, 4.0),
     # d = 256: 64-key tiles
     (2, 2, 1, 4000, 256, True, 0, 1.0),
     (1, 2, 3, 1500, 256, False, 7, 1.0),
