@@ -39,6 +39,9 @@ METRIC = "attn fwd TFLOP/s (bf16, N=512–16k, d=64/128) and % of B200 dense BF1
 DEFAULT_WORKLOAD = "B8_H16_N2048_d128_causal"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_BF16_TFLOPS = 2250.0
+# ex2.approx throughput measured on the B200: 16 per clock per SM (about
+# 8 cycles per warp instruction per sub-partition).
+EX2_PER_CLK_PER_SM = 16
 BWD_METRIC = "attn bwd TFLOP/s (bf16, FLOP = 2.5 x forward FLOP) and % of B200 dense BF16 peak"
 DECODE_METRIC = "split-K/V attn fwd effective HBM GB/s (Q,K,V read once, O,LSE written once)"
 KERNEL_SOURCES = ["exact_tiled_attention_45_b200/csrc/fa2_fwd.cu", "exact_tiled_attention_45_b200/csrc/sm100_ptx.cuh",
@@ -700,6 +703,20 @@ def main():
     total_flops = w.flops * world
     value = aggregate_tflops(w.flops, world, ms_per_step)
 
+    # Per-launch distribution, from a second pass of the same launches with
+    # an event pair around each (outside the bracketed timing above).
+    step_times = []
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in pairs:
+        if flush is not None:
+            flush.zero_()
+        a.record(stream)
+        fa2.fwd(q, k, v, causal=w.causal, out=o, lse=lse, stream=stream)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    step_times = sorted(a.elapsed_time(b) for a, b in pairs)
+    fa2.sync_status(stream)
+
     # End to end through the host-buffer entry point: pinned host inputs in,
     # host outputs back, copies inside the timed region.
     e2e = None
@@ -735,6 +752,22 @@ def main():
     achieved = w.flops / (kernel_ms * 1e-3) / 1e12
     src = source_hash()
     traffic = recorded_traffic(w.name, src)
+
+    def pct(p):
+        return step_times[min(len(step_times) - 1, int(round(p / 100.0 * (len(step_times) - 1))))]
+
+    clocks = sampler.summary()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    sm_hz = float(clocks.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    exp_ms = w.exps / (EX2_PER_CLK_PER_SM * sms * sm_hz) * 1e3
+    floors = {
+        "hbm_ms": w.io_bytes / (hbm * 1e9) * 1e3, "hbm_bytes": w.io_bytes,
+        "tensor_ms": w.flops / (peak * 1e12) * 1e3,
+        "exp_ms": exp_ms, "exps": w.exps,
+        "exp_basis": f"{EX2_PER_CLK_PER_SM} ex2/clk/SM x {sms} SMs x median SM clock (all exponentials on the MUFU)",
+        "exp_bound_pct": 100.0 * exp_ms / kernel_ms,
+    }
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         cpu, _ = cpu_oracle_sample(w, args.cpu_seconds, q_h, k_h, v_h)
@@ -755,7 +788,10 @@ def main():
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_kind} bf16 burst",
                      "kernel": "fa2_fwd_kernel", "src": src},
-        "clocks": sampler.summary(),
+        "step_ms": {"median": pct(50), "p10": pct(10), "p90": pct(90), "n": len(step_times),
+                    "pass": "second pass, one event pair per launch"},
+        "floors": floors,
+        "clocks": clocks,
         "gpu_launches": args.steps,
         "e2e": e2e,
         "cpu_baseline": cpu,

@@ -56,6 +56,17 @@ class Workload:
         f = 4.0 * self.B * self.H * self.N * self.N * self.d
         return f / 2 if self.causal else f
 
+    @property
+    def exps(self) -> float:
+        """Exponentials by the same convention: B*H*N^2, halved when causal."""
+        e = float(self.B * self.H) * self.N * self.N
+        return e / 2 if self.causal else e
+
+    @property
+    def io_bytes(self) -> float:
+        """Algorithmic HBM bytes: Q, K, V read once, O written (bf16), LSE written (fp32)."""
+        return float(self.B * self.H) * (8 * self.N * self.d + 4 * self.N)
+
     def as_dict(self) -> dict:
         return {"workload": self.name, "B": self.B, "H": self.H, "N": self.N,
                 "d": self.d, "causal": self.causal, "qk_mult": self.qk_mult}
