@@ -7,6 +7,8 @@ returned in bf16, and that final rounding alone can reach 2^-5 / 2 = 0.016 for
 are compared element by element; full-size workloads on sampled rows that
 include tile boundaries, the first and the last row.
 """
+import zlib
+
 import numpy as np
 import pytest
 import torch
@@ -140,6 +142,31 @@ def test_full_size_sampled_rows(name, mult):
                                             scale=w.d ** -0.5)
         assert_close(o_all[b, h, rows].double().numpy(), lse_all[b, h, rows].double().numpy(), o_ref, lse_ref,
                      f"{name} x{mult} head ({b},{h})")
+
+
+GRID = [f"grid_N{n}_d{d}_{c}" for d in (64, 128) for c in ("full", "causal")
+        for n in (512, 1024, 2048, 4096, 8192, 16384)] + ["grid_N2048_d256_causal", "grid_N16384_d256_full"]
+
+
+@pytest.mark.parametrize("name", GRID)
+@pytest.mark.parametrize("mult", [1.0, 4.0], ids=["x1", "x4"])
+def test_grid_point_sampled_rows(name, mult):
+    # Every point of the headline grid at full size (the launch the bench
+    # times): all outputs finite, one random head's sampled rows against the
+    # oracle.
+    w = WORKLOADS[name]
+    q, k, v = make_qkv(w.B, w.H, w.N, w.d, seed=0, qk_mult=mult)
+    o_d, lse_d = fwd(q.cuda(), k.cuda(), v.cuda(), causal=w.causal)
+    sync_status()
+    assert torch.isfinite(lse_d).all().item() and torch.isfinite(o_d.float()).all().item()
+    rng = np.random.default_rng(zlib.crc32(f"{name} {mult}".encode()))
+    b, h = int(rng.integers(w.B)), int(rng.integers(w.H))
+    rows = _sample_rows(w.N, rng, extra=4)
+    o_ref, lse_ref = attention_ref_rows(q[b:b + 1, h:h + 1].double().numpy(), k[b:b + 1, h:h + 1].double().numpy(),
+                                        v[b:b + 1, h:h + 1].double().numpy(), 0, 0, rows, causal=w.causal,
+                                        scale=w.d ** -0.5)
+    assert_close(o_d[b, h, rows].double().cpu().numpy(), lse_d[b, h, rows].double().cpu().numpy(), o_ref, lse_ref,
+                 f"{name} x{mult} head ({b},{h})")
 
 
 def test_constant_v_gives_constant_output():
