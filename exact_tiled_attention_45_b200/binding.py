@@ -143,7 +143,8 @@ def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
     """End-to-end call on HOST tensors (pinned for full copy bandwidth).
 
     Copies q, k, v to the device, runs the kernel, copies O and LSE back and
-    returns after they have landed.  ``workspace`` is an optional uint8 CUDA
+    returns after they have landed (the library overlaps the copies and the
+    kernels over chunks of heads).  Outputs are allocated pinned when q is.  ``workspace`` is an optional uint8 CUDA
     tensor of at least :func:`workspace_bytes` bytes, reused across calls.
     """
     lib = load()
@@ -156,10 +157,11 @@ def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
         workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
     if workspace.numel() < need:
         raise ValueError(f"workspace needs {need} bytes")
+    pinned = q.is_pinned()
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=pinned)
     if lse is None:
-        lse = torch.empty((B, H, N), dtype=torch.float32)
+        lse = torch.empty((B, H, N), dtype=torch.float32, pin_memory=pinned)
     st = lib.fa2_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                           B, H, N, d, int(bool(causal)), float(scale), workspace.data_ptr(),
                           workspace.numel(), _stream_handle(stream))

@@ -675,6 +675,44 @@ static int make_tmap(CUtensorMap* tm, const void* ptr, int d, int N, int BH, int
   return FA2_OK;
 }
 
+// Streams and events of the host-buffer entry point, created once per device
+// on first use and kept for the life of the process; the mutex serialises
+// calls that share them (each call returns only after its work has landed).
+struct HostPipe {
+  static constexpr int MAX_CHUNKS = 8;
+  std::mutex mu;
+  cudaStream_t compute = nullptr, download = nullptr;
+  cudaEvent_t uploaded[MAX_CHUNKS] = {}, computed[MAX_CHUNKS] = {}, drained = nullptr;
+};
+
+static int host_pipe(HostPipe** out) {
+  constexpr int MAX_DEVICES = 64;
+  static HostPipe pipes[MAX_DEVICES];
+  static std::once_flag once[MAX_DEVICES];
+  static int created[MAX_DEVICES] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) {
+    set_detail("no usable current device");
+    return FA2_ERR_CUDA;
+  }
+  std::call_once(once[dev], [dev] {
+    HostPipe& p = pipes[dev];
+    bool ok = cudaStreamCreateWithFlags(&p.compute, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&p.download, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&p.drained, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; ok && i < HostPipe::MAX_CHUNKS; ++i)
+      ok = cudaEventCreateWithFlags(&p.uploaded[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&p.computed[i], cudaEventDisableTiming) == cudaSuccess;
+    created[dev] = ok ? 1 : -1;
+  });
+  if (created[dev] != 1) {
+    set_detail("could not create the host pipeline's streams and events");
+    return FA2_ERR_CUDA;
+  }
+  *out = &pipes[dev];
+  return FA2_OK;
+}
+
 static bool overlap(const void* a, size_t na, const void* b, size_t nb) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
   return x < y + nb && y < x + na;
@@ -1212,23 +1250,79 @@ int fa2_fwd_host(const void* q, const void* k, const void* v, void* o, float* ls
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t tb = static_cast<size_t>(B) * H * N * d * 2;
   const size_t t = (tb + 255) & ~static_cast<size_t>(255);
-  const size_t lb = static_cast<size_t>(B) * H * N * 4;
   char* ws = static_cast<char*>(workspace);
-  void *dq = ws, *dk = ws + t, *dv = ws + 2 * t, *dout = ws + 3 * t;
+  char *dq = ws, *dk = ws + t, *dv = ws + 2 * t, *dout = ws + 3 * t;
   float* dl = reinterpret_cast<float*>(ws + 4 * t);
-  cudaError_t e;
-  if ((e = cudaMemcpyAsync(dq, q, tb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(dk, k, tb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(dv, v, tb, cudaMemcpyHostToDevice, s)) != cudaSuccess) {
-    fa2::set_detail("host-to-device copy: %s", cudaGetErrorString(e));
-    return FA2_ERR_CUDA;
+  // Validate once on the whole shape before any copy is queued.
+  {
+    const int st = fa2::validate(dq, dk, dv, dout, dl, B, H, N, d, scale);
+    if (st != FA2_OK) return st;
   }
-  int st = fa2_fwd(dq, dk, dv, dout, dl, B, H, N, d, causal, scale, stream);
-  if (st != FA2_OK) return st;
-  if ((e = cudaMemcpyAsync(o, dout, tb, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(lse, dl, lb, cudaMemcpyDeviceToHost, s)) != cudaSuccess) {
-    fa2::set_detail("device-to-host copy: %s", cudaGetErrorString(e));
-    return FA2_ERR_CUDA;
+  fa2::HostPipe* pipe = nullptr;
+  {
+    const int st = fa2::host_pipe(&pipe);
+    if (st != FA2_OK) return st;
+  }
+  std::lock_guard<std::mutex> lock(pipe->mu);
+  // The B*H heads are contiguous ([B, H, N, d]), so a run of heads is one
+  // contiguous slice of every tensor.  Chunk c is uploaded on the caller's
+  // stream, computed on the pipe's compute stream once its upload is done, and
+  // downloaded on the pipe's download stream once computed: the copies of
+  // neighbouring chunks overlap each other (both copy directions) and the
+  // kernels.  Every head is computed exactly as in one whole call.
+  // Chunks are runs of whole batches when there are enough batches (each
+  // chunk then keeps the caller's H), else runs of heads (each shorter than H).
+  const long long BH = static_cast<long long>(B) * H;
+  const int chunks = static_cast<int>(std::min<long long>(fa2::HostPipe::MAX_CHUNKS, BH));
+  const bool by_batch = B >= chunks;
+  const size_t head_b = static_cast<size_t>(N) * d * 2, head_l = static_cast<size_t>(N) * 4;
+  cudaError_t e = cudaSuccess;
+  int st = FA2_OK;
+  int c = 0;
+  for (; c < chunks; ++c) {
+    const long long u0 = (by_batch ? B : BH) * c / chunks, u1 = (by_batch ? B : BH) * (c + 1) / chunks;
+    const long long h0 = by_batch ? u0 * H : u0, h1 = by_batch ? u1 * H : u1;
+    const int cB = by_batch ? static_cast<int>(u1 - u0) : 1, cH = by_batch ? H : static_cast<int>(u1 - u0);
+    const size_t ob = static_cast<size_t>(h0) * head_b, nb = static_cast<size_t>(h1 - h0) * head_b;
+    const size_t ol = static_cast<size_t>(h0) * head_l, nl = static_cast<size_t>(h1 - h0) * head_l;
+    if ((e = cudaMemcpyAsync(dq + ob, static_cast<const char*>(q) + ob, nb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(dk + ob, static_cast<const char*>(k) + ob, nb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(dv + ob, static_cast<const char*>(v) + ob, nb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+        (e = cudaEventRecord(pipe->uploaded[c], s)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(pipe->compute, pipe->uploaded[c], 0)) != cudaSuccess) {
+      fa2::set_detail("host-to-device copy: %s", cudaGetErrorString(e));
+      st = FA2_ERR_CUDA;
+      break;
+    }
+    st = fa2_fwd(dq + ob, dk + ob, dv + ob, dout + ob, dl + h0 * N, cB, cH, N, d, causal, scale, pipe->compute);
+    if (st != FA2_OK) break;
+    if ((e = cudaEventRecord(pipe->computed[c], pipe->compute)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(pipe->download, pipe->computed[c], 0)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(static_cast<char*>(o) + ob, dout + ob, nb, cudaMemcpyDeviceToHost, pipe->download)) !=
+            cudaSuccess ||
+        (e = cudaMemcpyAsync(reinterpret_cast<char*>(lse) + ol, reinterpret_cast<char*>(dl) + ol, nl,
+                             cudaMemcpyDeviceToHost, pipe->download)) != cudaSuccess) {
+      fa2::set_detail("device-to-host copy: %s", cudaGetErrorString(e));
+      st = FA2_ERR_CUDA;
+      break;
+    }
+  }
+  // The caller's stream is ordered after everything queued on the pipe's
+  // streams (also on an error part-way), so its synchronisation covers them.
+  if ((e = cudaEventRecord(pipe->drained, pipe->download)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(s, pipe->drained, 0)) != cudaSuccess ||
+      (e = cudaEventRecord(pipe->drained, pipe->compute)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(s, pipe->drained, 0)) != cudaSuccess) {
+    cudaStreamSynchronize(pipe->compute);
+    cudaStreamSynchronize(pipe->download);
+    if (st == FA2_OK) {
+      fa2::set_detail("stream ordering: %s", cudaGetErrorString(e));
+      st = FA2_ERR_CUDA;
+    }
+  }
+  if (st != FA2_OK) {
+    cudaStreamSynchronize(s);
+    return st;
   }
   return fa2_sync_status(stream);
 }

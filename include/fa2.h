@@ -76,8 +76,14 @@ int fa2_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
  * written to host memory, and the call returns after the results have landed.
  * `workspace` is a caller-owned device buffer of at least
  * fa2_fwd_host_workspace_bytes(B,H,N,d) bytes, 256-byte aligned, that holds
- * the device copies.  Returns FA2_ERR_TIMEOUT if the kernel reported a
- * timeout.
+ * the device copies.  The work is split into up to 8 chunks of whole batches
+ * (or of heads when B < 8): uploads run on `stream`, each chunk's kernel on a
+ * compute stream and its downloads on a download stream of the library's own
+ * (created once per device on first use, kept until the process ends), so
+ * copies in both directions overlap the kernels; results are identical to
+ * one fa2_fwd call.  Concurrent calls on one device are serialised.  Returns
+ * FA2_ERR_TIMEOUT if a kernel reported a timeout; after any error every
+ * queued copy and kernel has completed before the call returns.
  */
 int fa2_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                  int causal, float scale, void* workspace, size_t workspace_bytes, void* stream);

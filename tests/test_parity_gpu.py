@@ -199,6 +199,21 @@ def test_repeatable_bitwise():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("B,H,N,d,causal", [(9, 2, 300, 64, True), (3, 5, 257, 128, False), (1, 3, 129, 96, True),
+                                         (2, 1, 200, 256, True)],
+                         ids=["by-batch", "by-head", "three-heads", "d256"])
+def test_host_entry_chunks_match_device_call(B, H, N, d, causal):
+    # The host entry point uploads, computes and downloads in chunks of whole
+    # batches (B >= chunks) or of heads; every head is computed as in one call.
+    q, k, v = make_qkv(B, H, N, d, seed=9)
+    o1, l1 = fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+    sync_status()
+    o2, l2 = fwd_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), causal=causal)
+    assert torch.equal(o1.cpu(), o2) and torch.equal(l1.cpu(), l2)
+    o3, l3 = fwd_host(q, k, v, causal=causal)  # pageable host memory
+    assert torch.equal(o2, o3) and torch.equal(l2, l3)
+
+
 def test_side_stream_and_host_entry_agree():
     q, k, v = make_qkv(2, 2, 640, 64, seed=8)
     s = torch.cuda.Stream()
