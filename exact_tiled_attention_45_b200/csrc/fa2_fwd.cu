@@ -898,11 +898,11 @@ static size_t skv_workspace_bytes(int B, int H, int Nq, int d, int splits) {
   return round256(rows * d * 4) + round256(rows * 4);
 }
 
-template <int HD, bool CAUSAL>
+template <int HD, bool CAUSAL, bool QUAD>
 static int skv_launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const SkvParams& prm,
                         int n_q_tiles, int splits, __nv_bfloat16* o, float* lse, cudaStream_t stream) {
   using C = SkvCfg<HD>;
-  auto kern = fa2_splitkv_kernel<HD, CAUSAL>;
+  auto kern = fa2_splitkv_kernel<HD, CAUSAL, QUAD>;
   static int attr_done_mask = 0;  // per device bit (devices 0..31)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -979,9 +979,11 @@ static int splitkv_impl(const void* q, const void* k, const void* v, void* o, fl
     set_detail("output or workspace buffers overlap inputs or each other");
     return FA2_ERR_INVALID_ARG;
   }
+  // Quarter mode for at most 32 query rows (d <= 128): 32-row query boxes.
+  const bool quad = Nq <= 32 && padded_hd(d) <= 128;
   CUtensorMap tq, tk, tv;
   int st;
-  if ((st = make_tmap(&tq, q, d, Nq, static_cast<int>(BH))) != FA2_OK) return st;
+  if ((st = make_tmap(&tq, q, d, Nq, static_cast<int>(BH), quad ? 32 : 128)) != FA2_OK) return st;
   if ((st = make_tmap(&tk, k, d, Nk, static_cast<int>(BH), skv_tile_keys(d))) != FA2_OK) return st;
   if ((st = make_tmap(&tv, v, d, Nk, static_cast<int>(BH), skv_tile_keys(d))) != FA2_OK) return st;
   SkvParams prm;
@@ -1002,14 +1004,21 @@ static int splitkv_impl(const void* q, const void* k, const void* v, void* o, fl
   prm.timeout_ns = DEFAULT_TIMEOUT_NS;
   const int n_q_tiles = (Nq + BM - 1) / BM;
   auto* ob = static_cast<__nv_bfloat16*>(o);
-  if (padded_hd(d) == 64)
-    return causal ? skv_launch_t<64, true>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
-                  : skv_launch_t<64, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
+  if (padded_hd(d) == 64) {
+    if (quad)
+      return causal ? skv_launch_t<64, true, true>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
+                    : skv_launch_t<64, false, true>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
+    return causal ? skv_launch_t<64, true, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
+                  : skv_launch_t<64, false, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
+  }
   if (padded_hd(d) == 256)
-    return causal ? skv_launch_t<256, true>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
-                  : skv_launch_t<256, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
-  return causal ? skv_launch_t<128, true>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
-                : skv_launch_t<128, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
+    return causal ? skv_launch_t<256, true, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
+                  : skv_launch_t<256, false, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
+  if (quad)
+    return causal ? skv_launch_t<128, true, true>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
+                  : skv_launch_t<128, false, true>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
+  return causal ? skv_launch_t<128, true, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream)
+                : skv_launch_t<128, false, false>(tq, tk, tv, prm, n_q_tiles, splits, ob, lse, stream);
 }
 
 // ------------------------------------------------------------------ backward host side

@@ -23,6 +23,16 @@
 // computed while the softmax works on the current one), a separate P buffer,
 // and O.  Rows past Nq are computed on zero queries and never stored.
 //
+// Quarter mode (QUAD, at most 32 query rows, d <= 128): the query rows are
+// loaded four times, into TMEM lane quadrants 0, 32, 64 and 96, so every
+// softmax warp holds all of them, and warp w takes key columns 32w..32w+31 of
+// each tile: a quarter of the exponentials per warp instead of all 128
+// columns on the one warp whose lanes hold the rows.  Each warp keeps its own
+// running max and sum; its P row is zero outside its key columns, so PV
+// accumulates in quadrant w exactly the partial output of those keys.  At the
+// end the four partials merge exactly (the same formula as the ranges) through
+// shared memory.
+//
 // Head dimension 256 (also served to the square entry point as one range with
 // Nq = Nk): 64-key tiles, so that a 256-column O accumulator, two score
 // buffers and P fit the 512 TMEM columns and two stages of K and V fit shared
@@ -85,11 +95,12 @@ struct SkvBarriers {
 };
 static_assert(sizeof(SkvBarriers) <= 256, "barrier block");
 
-template <int HD, bool CAUSAL>
+template <int HD, bool CAUSAL, bool QUAD>
 __global__ void __launch_bounds__(SKV_THREADS, 1)
     fa2_splitkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const SkvParams p) {
   using C = SkvCfg<HD>;
+  static_assert(!QUAD || C::SBN == 128, "quarter mode needs 128-key tiles");
   const int q_first = static_cast<int>(blockIdx.x) * BM;
   const int bh = static_cast<int>(blockIdx.y);
   const int split = static_cast<int>(blockIdx.z);
@@ -172,7 +183,14 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       mbar_arrive_expect_tx(b_q, C::Q_BYTES);
-      for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * C::Q_CHUNK, &tm_q, b_q, c * 64, q_first, bh);
+      if constexpr (QUAD) {
+        // Four copies of the (at most 32) query rows, 32-row boxes, at rows
+        // 0, 32, 64, 96 of the tile; rows past Nq are zero-filled.
+        for (int w = 0; w < 4; ++w)
+          for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * C::Q_CHUNK + w * 32 * 128, &tm_q, b_q, c * 64, 0, bh);
+      } else {
+        for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * C::Q_CHUNK, &tm_q, b_q, c * 64, q_first, bh);
+      }
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < nkv; ++j) {
         const int kv0 = (kt_begin + j) * C::SBN;
@@ -245,6 +263,190 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
       }
       mma_commit(b_final);
       wait_drain(b_final, 0, to);
+    }
+  } else if constexpr (QUAD) {
+    // ------------------------------------------------------------ softmax warps 0..3, quarter mode
+    const int qrow = lane;  // query row of this thread (each warp holds a copy)
+    const int pos = offset + qrow;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int col0 = warp * 32;  // this warp's key columns of every tile
+    const float c_log2 = p.scale_log2;
+    const uint64_t cc = f2_pack(c_log2, c_log2);
+    {
+      // P of the other warps' keys stays zero in this warp's lanes.
+      uint32_t z[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) z[e] = 0u;
+      tmem_st32(lane_addr + C::TM_P, z);
+      tmem_st32(lane_addr + C::TM_P + 32, z);
+      tmem_wait_st();
+    }
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int i = 0; i < nkv; ++i) {
+      const int sb = i & 1;
+      ok = wait_warp(smem_u32(&bars->s_full[sb]), (i >> 1) & 1, abort_flag, to);
+      if (!ok) break;
+      tc_fence_after();
+      const int kv0 = (kt_begin + i) * C::SBN + col0;
+      uint32_t s[32];
+      tmem_ld32(lane_addr + (sb ? C::TM_S1 : C::TM_S0) + col0, s);
+      tmem_wait_ld();
+      reg_fence32(s);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[sb]));
+      const int lim = CAUSAL ? min(pos, p.Nk - 1) - kv0 : p.Nk - 1 - kv0;
+      if (lim < 31) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (e > lim) s[e] = __float_as_uint(-INFINITY);
+      }
+      float mx4[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) mx4[a] = __uint_as_float(s[a]);
+#pragma unroll
+      for (int e = 4; e + 8 <= 32; e += 8)  // columns 4 .. 27
+#pragma unroll
+        for (int a = 0; a < 4; ++a) mx4[a] = fmax3(mx4[a], __uint_as_float(s[e + a]), __uint_as_float(s[e + 4 + a]));
+#pragma unroll
+      for (int a = 0; a < 4; ++a) mx4[a] = fmaxf(mx4[a], __uint_as_float(s[28 + a]));  // the last 4
+      const float mx = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
+      const float m_cand = mx * c_log2;
+      float m_new = m;
+      if (m_cand > m + RESCALE_THRESHOLD) m_new = m_cand;
+      const bool rescale = (i > 0) && (m_new != m);
+      const float alpha = rescale ? ex2(m - m_new) : 1.f;
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      const uint64_t mm = f2_pack(-m_use, -m_use);
+      uint64_t acc[4] = {0, 0, 0, 0};
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), cc, mm);
+        float x0, x1;
+        f2_unpack(x, x0, x1);
+        const float p0 = ex2(x0), p1 = ex2(x1);
+        acc[(e >> 1) & 3] = f2_add(acc[(e >> 1) & 3], f2_pack(p0, p1));
+        pk[e >> 1] = pack_bf16x2(p0, p1);
+      }
+      float r0, r1, r2, r3;
+      f2_unpack(f2_add(acc[0], acc[1]), r0, r1);
+      f2_unpack(f2_add(acc[2], acc[3]), r2, r3);
+      const float rowsum = (r0 + r1) + (r2 + r3);
+      if (i > 0) {
+        // O and the P buffer are in use by PV(i-1) until it completes.
+        ok = wait_warp(b_pv, (i - 1) & 1, abort_flag, to);
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale)) {
+          const uint64_t aa = f2_pack(alpha, alpha);
+#pragma unroll
+          for (int c = 0; c < HD / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + C::TM_O + c * 32, o);
+            tmem_wait_ld();
+            reg_fence32(o);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float a0, a1;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), aa), a0, a1);
+              o[e] = __float_as_uint(a0);
+              o[e + 1] = __float_as_uint(a1);
+            }
+            tmem_st32(lane_addr + C::TM_O + c * 32, o);
+          }
+        }
+      }
+      tmem_st16(lane_addr + C::TM_P + 16 * warp, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_p);
+      l = l * alpha + rowsum;
+      m = m_new;
+    }
+    if (ok) ok = wait_warp(b_pv, (nkv - 1) & 1, abort_flag, to);
+    // Merge of the four quarters.  Every softmax warp reaches both named
+    // barriers whatever happened above (after a time-out the values are
+    // unspecified, as documented, but no warp is left waiting).  The K ring
+    // is idle here: its last reader, an S MMA, completed before the final PV.
+    constexpr int OST = HD + 4;  // padded row stride (floats) of the exchange buffer
+    float* xo = reinterpret_cast<float*>(smem + C::OFF_K);  // [4 warps][32 rows][OST]
+    float* xm = reinterpret_cast<float*>(smem + C::OFF_V);  // [4][32] running max (log2)
+    float* xl = xm + 128;                                   // [4][32] running sum
+    static_assert(4 * 32 * OST * 4 <= C::KS * C::KV_BYTES, "exchange buffer");
+    xm[warp * 32 + lane] = m;
+    xl[warp * 32 + lane] = l;
+    named_barrier(1, 128);
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, xm[w * 32 + lane]);
+    float L = 0.f, wt_self = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float mw = xm[w * 32 + lane];
+      const float wt = (mw == -INFINITY) ? 0.f : ex2(mw - M);
+      L += wt * xl[w * 32 + lane];
+      if (w == warp) wt_self = wt;
+    }
+    const float f_self = (L > 0.f) ? wt_self / L : 0.f;
+    tc_fence_after();
+#pragma unroll
+    for (int c = 0; c < HD / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld32(lane_addr + C::TM_O + c * 32, o);
+      tmem_wait_ld();
+      reg_fence32(o);
+      float4* dst = reinterpret_cast<float4*>(xo + (warp * 32 + lane) * OST + c * 32);
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        dst[e / 4] = make_float4(__uint_as_float(o[e]) * f_self, __uint_as_float(o[e + 1]) * f_self,
+                                 __uint_as_float(o[e + 2]) * f_self, __uint_as_float(o[e + 3]) * f_self);
+    }
+    named_barrier(1, 128);
+    if (ok && qrow < p.Nq) {
+      // Warp w sums columns [w*HD/4, (w+1)*HD/4) of this thread's row.
+      constexpr int CW = HD / 4;
+      const int cb = warp * CW;
+      const size_t prow = (static_cast<size_t>(split) * p.BH + bh) * p.Nq + qrow;
+#pragma unroll
+      for (int c = 0; c < CW; c += 8) {
+        float v8[8];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const float4 b = *reinterpret_cast<const float4*>(xo + (w * 32 + qrow) * OST + cb + c + 4 * h);
+            a.x += b.x;
+            a.y += b.y;
+            a.z += b.z;
+            a.w += b.w;
+          }
+          v8[4 * h] = a.x;
+          v8[4 * h + 1] = a.y;
+          v8[4 * h + 2] = a.z;
+          v8[4 * h + 3] = a.w;
+        }
+        if (p.direct) {
+          if (cb + c < p.d)
+            *reinterpret_cast<uint4*>(p.o + prow * p.d + cb + c) =
+                make_uint4(pack_bf16x2(v8[0], v8[1]), pack_bf16x2(v8[2], v8[3]), pack_bf16x2(v8[4], v8[5]),
+                           pack_bf16x2(v8[6], v8[7]));
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.o_part + prow * HD + cb + c);
+          dst[0] = make_float4(v8[0], v8[1], v8[2], v8[3]);
+          dst[1] = make_float4(v8[4], v8[5], v8[6], v8[7]);
+        }
+      }
+      if (warp == 0) {
+        const float lse_row = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+        if (p.direct)
+          p.lse[prow] = lse_row;
+        else
+          p.lse_part[prow] = lse_row;
+      }
     }
   } else {
     // ------------------------------------------------------------ softmax warps 0..3

@@ -75,6 +75,12 @@ CASES = [
     (1, 2, 4, 4, 256, True, 0, 1.0),
     (2, 1, 3, 33, 128, True, 2, 4.0),
     (1, 2, 1, 20000, 64, True, 0, 4.0),
+    # quarter mode (at most 32 query rows, d <= 128) at its edges
+    (1, 2, 32, 2000, 128, True, 0, 1.0),
+    (2, 1, 32, 33, 64, True, 3, 4.0),
+    (1, 2, 33, 2000, 128, True, 0, 1.0),     # one row too many: the full-tile mode
+    (1, 1, 31, 4096, 96, False, 2, 1.0),
+    (3, 2, 1, 95, 32, True, 0, 1.0),         # fewer keys than one warp's quarter of a tile
     # d = 256: 64-key tiles
     (2, 2, 1, 4000, 256, True, 0, 1.0),
     (1, 2, 3, 1500, 256, False, 7, 1.0),
