@@ -118,7 +118,10 @@ int fa2_fwd_inject_timeout(const void* q, const void* k, const void* v, void* o,
  * idle, so the keys are split into ranges: one CTA per (128-row query tile,
  * batch*head, key range) computes that range's partial output and
  * logsumexp, and a second kernel merges them exactly
- * (LSE = ln sum_r exp(LSE_r), O = sum_r exp(LSE_r - LSE) O_r).
+ * (LSE = ln sum_r exp(LSE_r), O = sum_r exp(LSE_r - LSE) O_r).  With at
+ * most 32 query rows and d <= 128 the same split is also applied inside each
+ * CTA: every softmax warp takes a quarter of each key tile for all the rows
+ * and the four quarters merge exactly before the range result is written.
  *
  *   q       : device pointer, bf16 [B,H,Nq,d], contiguous, 16-byte aligned.
  *   k, v    : device pointers, bf16 [B,H,Nk,d], contiguous, 16-byte aligned.
