@@ -106,6 +106,24 @@ def _check_qkv(q, k, v, device: str):
         raise ValueError("q, k, v must share the shape [B, H, N, d]")
 
 
+def _check_buffer(name: str, t: torch.Tensor, shape, dtype, device: str) -> None:
+    """A caller-provided output or workspace buffer the kernels will write."""
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device.type != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+
+
+def _check_workspace(workspace: torch.Tensor, need: int) -> None:
+    _check_buffer("workspace", workspace, None, torch.uint8, "cuda")
+    if workspace.numel() < need:
+        raise ValueError(f"workspace needs {need} bytes, got {workspace.numel()}")
+
+
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, scale: float | None = None,
         out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
     """Exact attention forward on CUDA tensors.  Returns (O bf16, LSE fp32).
@@ -121,6 +139,8 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check_buffer("out", out, q.shape, torch.bfloat16, "cuda")
+    _check_buffer("lse", lse, (B, H, N), torch.float32, "cuda")
     st = lib.fa2_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                      B, H, N, d, int(bool(causal)), float(scale), _stream_handle(stream))
     _check(st, lib)
@@ -144,8 +164,9 @@ def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
 
     Copies q, k, v to the device, runs the kernel, copies O and LSE back and
     returns after they have landed (the library overlaps the copies and the
-    kernels over chunks of heads).  Outputs are allocated pinned when q is.  ``workspace`` is an optional uint8 CUDA
-    tensor of at least :func:`workspace_bytes` bytes, reused across calls.
+    kernels over chunks of heads).  Outputs are allocated pinned when q is.
+    ``workspace`` is an optional uint8 CUDA tensor of at least
+    :func:`workspace_bytes` bytes, reused across calls.
     """
     lib = load()
     _check_qkv(q, k, v, "cpu")
@@ -155,13 +176,14 @@ def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
     need = workspace_bytes(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
-    if workspace.numel() < need:
-        raise ValueError(f"workspace needs {need} bytes")
+    _check_workspace(workspace, need)
     pinned = q.is_pinned()
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, pin_memory=pinned)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, pin_memory=pinned)
+    _check_buffer("out", out, q.shape, torch.bfloat16, "cpu")
+    _check_buffer("lse", lse, (B, H, N), torch.float32, "cpu")
     st = lib.fa2_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                           B, H, N, d, int(bool(causal)), float(scale), workspace.data_ptr(),
                           workspace.numel(), _stream_handle(stream))
@@ -235,11 +257,15 @@ def fwd_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool 
     need = splitkv_workspace_bytes(B, H, Nq, Nk, d, n_splits)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is not None:
+        _check_workspace(workspace, need)
     ws_ptr, ws_len = (workspace.data_ptr(), workspace.numel()) if workspace is not None else (None, 0)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _check_buffer("out", out, q.shape, torch.bfloat16, "cuda")
+    _check_buffer("lse", lse, (B, H, Nq), torch.float32, "cuda")
     st = lib.fa2_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                              B, H, Nq, Nk, d, int(bool(causal)), float(scale), int(n_splits),
                              ws_ptr, ws_len, _stream_handle(stream))
@@ -272,6 +298,8 @@ def fwd_splitkv_static(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _check_buffer("out", out, q.shape, torch.bfloat16, "cuda")
+    _check_buffer("lse", lse, (B, H, Nq), torch.float32, "cuda")
     st = lib.fa2_fwd_splitkv_static(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                     B, H, Nq, Nk, d, int(bool(causal)), float(scale), int(n_splits),
                                     _stream_handle(stream))
@@ -305,9 +333,12 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse:
     need = bwd_workspace_bytes(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check_workspace(workspace, need)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_buffer(name, t, q.shape, torch.bfloat16, "cuda")
     st = lib.fa2_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
                      workspace.data_ptr(), workspace.numel(), _stream_handle(stream))

@@ -262,3 +262,26 @@ def test_head_dim_256_uses_64_key_tiles(lib):
     assert lib.fa2_fwd_splitkv_splits(1, 1, 1, 1000, 256, 0) == 4
     rows = 2 * 1 * 2 * 3
     assert lib.fa2_fwd_splitkv_workspace_bytes(1, 2, 3, 1000, 256, 2) == (rows * 256 * 4 + 255) // 256 * 256 + 256
+
+
+def test_output_buffer_checks_reject_wrong_buffers():
+    # Caller-provided outputs and workspaces are checked before the library
+    # sees their pointers (a short or misshapen buffer would be written past
+    # its end by the kernels).
+    import torch
+    ok = torch.empty((2, 3, 5, 64), dtype=torch.bfloat16)
+    binding._check_buffer("out", ok, (2, 3, 5, 64), torch.bfloat16, "cpu")
+    with pytest.raises(TypeError):
+        binding._check_buffer("out", ok.float(), (2, 3, 5, 64), torch.bfloat16, "cpu")
+    with pytest.raises(ValueError):
+        binding._check_buffer("out", ok[:, :, :4], (2, 3, 5, 64), torch.bfloat16, "cpu")
+    with pytest.raises(ValueError):
+        binding._check_buffer("out", ok.transpose(2, 3).contiguous().transpose(2, 3), (2, 3, 5, 64),
+                              torch.bfloat16, "cpu")
+    with pytest.raises(ValueError):
+        binding._check_buffer("out", ok, (2, 3, 5, 64), torch.bfloat16, "cuda")
+    lse = torch.empty((2, 3, 5), dtype=torch.float32)
+    with pytest.raises(ValueError):
+        binding._check_buffer("lse", lse, (2, 3, 6), torch.float32, "cpu")
+    with pytest.raises(ValueError):
+        binding._check_workspace(torch.empty(16, dtype=torch.uint8), 16)  # host memory, not device
