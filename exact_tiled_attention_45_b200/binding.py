@@ -21,9 +21,9 @@ FA2_OK, FA2_ERR_INVALID_ARG, FA2_ERR_UNSUPPORTED, FA2_ERR_CUDA, FA2_ERR_TIMEOUT 
 
 #: Every symbol the header declares.
 EXPORTS = ("fa2_fwd", "fa2_fwd_host", "fa2_fwd_host_workspace_bytes", "fa2_sync_status",
-           "fa2_fwd_inject_timeout", "fa2_fwd_splitkv", "fa2_fwd_splitkv_splits",
+           "fa2_fwd_inject_timeout", "fa2_fwd_splitkv", "fa2_fwd_splitkv_inject_timeout", "fa2_fwd_splitkv_splits",
            "fa2_fwd_splitkv_workspace_bytes", "fa2_fwd_splitkv_static", "fa2_bwd", "fa2_bwd_workspace_bytes",
-           "fa2_strerror", "fa2_last_error_detail", "fa2_version")
+           "fa2_bwd_inject_timeout", "fa2_strerror", "fa2_last_error_detail", "fa2_version")
 
 _lib = None
 
@@ -52,6 +52,9 @@ def load() -> ctypes.CDLL:
     lib.fa2_fwd_splitkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _float, _int, _vp,
                                     ctypes.c_size_t, _vp]
     lib.fa2_fwd_splitkv.restype = _int
+    lib.fa2_fwd_splitkv_inject_timeout.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int,
+                                                   _float, _int, _vp, ctypes.c_size_t, ctypes.c_ulonglong, _vp]
+    lib.fa2_fwd_splitkv_inject_timeout.restype = _int
     lib.fa2_fwd_splitkv_splits.argtypes = [_int] * 6
     lib.fa2_fwd_splitkv_splits.restype = _int
     lib.fa2_fwd_splitkv_workspace_bytes.argtypes = [_int] * 6
@@ -63,6 +66,9 @@ def load() -> ctypes.CDLL:
     lib.fa2_bwd.restype = _int
     lib.fa2_bwd_workspace_bytes.argtypes = [_int] * 4
     lib.fa2_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.fa2_bwd_inject_timeout.argtypes = [_vp] * 9 + [_int] * 5 + [_float, _vp, ctypes.c_size_t, _int,
+                                                                     ctypes.c_ulonglong, _vp]
+    lib.fa2_bwd_inject_timeout.restype = _int
     lib.fa2_strerror.argtypes = [_int]
     lib.fa2_strerror.restype = ctypes.c_char_p
     lib.fa2_last_error_detail.argtypes = []
@@ -273,6 +279,31 @@ def fwd_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool 
     return out, lse
 
 
+def fwd_splitkv_inject_timeout(q, k, v, causal=False, scale=None, n_splits: int = 0, timeout_ns: int = 50_000_000,
+                               stream=None):
+    """Failure-path test hook of :func:`fwd_splitkv`: the range kernel runs
+    with its query load withheld (the merge still runs when there are two or
+    more key ranges).  Returns the status of :func:`sync_status` (expected
+    FA2_ERR_TIMEOUT)."""
+    lib = load()
+    _check_q_kv(q, k, v)
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = splitkv_workspace_bytes(B, H, Nq, Nk, d, n_splits)
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device) if need > 0 else None
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    h = _stream_handle(stream)
+    st = lib.fa2_fwd_splitkv_inject_timeout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                            lse.data_ptr(), B, H, Nq, Nk, d, int(bool(causal)), float(scale),
+                                            int(n_splits), ws.data_ptr() if ws is not None else None,
+                                            need, int(timeout_ns), h)
+    _check(st, lib)
+    return lib.fa2_sync_status(h)
+
+
 #: Bytes of the library's own scratch array used by :func:`fwd_splitkv_static`.
 SPLITKV_STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -344,3 +375,26 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse:
                      workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
     _check(st, lib)
     return dq, dk, dv
+
+
+def bwd_inject_timeout(q, k, v, o, lse, dout, kernel: int, causal: bool = False, scale=None,
+                       timeout_ns: int = 50_000_000, stream=None):
+    """Failure-path test hook of :func:`bwd`: ``kernel`` 0 withholds the dQ
+    kernel's Q/dO load, 1 the dK/dV kernel's K/V load.  Returns the status of
+    :func:`sync_status` (expected FA2_ERR_TIMEOUT)."""
+    lib = load()
+    _check_qkv(q, k, v, "cuda")
+    _check_qkv(o, dout, q, "cuda")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = bwd_workspace_bytes(B, H, N, d)
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    h = _stream_handle(stream)
+    st = lib.fa2_bwd_inject_timeout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                                    lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
+                                    int(bool(causal)), float(scale), ws.data_ptr(), ws.numel(), int(kernel),
+                                    int(timeout_ns), h)
+    _check(st, lib)
+    return lib.fa2_sync_status(h)

@@ -77,6 +77,9 @@ struct BwdParams {
   float scale;
   float scale_log2;
   unsigned long long timeout_ns;
+  // Test hook: 1 withholds the dQ kernel's Q/dO load, 2 the dK/dV kernel's
+  // K/V load, so that kernel's waits on it run out.
+  int inject_timeout;
 };
 
 // Work item of a 1-D grid: heads in groups of group_heads, tile rank the slow
@@ -200,10 +203,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   if (warp == BWD_PRODUCER_WARP) {
     if (lane == 0) {
       const uint32_t bq = smem_u32(&bars->qdo_full);
-      mbar_arrive_expect_tx(bq, 2 * C::TILE_BYTES);
-      for (int c = 0; c < C::KCH; ++c) {
-        tma_load_3d(sQ + c * C::CHUNK_BYTES, &tm_q, bq, c * 64, q0, bh);
-        tma_load_3d(sDO + c * C::CHUNK_BYTES, &tm_do, bq, c * 64, q0, bh);
+      const bool load_qdo = p.inject_timeout != 1;
+      if (load_qdo) {
+        mbar_arrive_expect_tx(bq, 2 * C::TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c) {
+          tma_load_3d(sQ + c * C::CHUNK_BYTES, &tm_q, bq, c * 64, q0, bh);
+          tma_load_3d(sDO + c * C::CHUNK_BYTES, &tm_do, bq, c * 64, q0, bh);
+        }
       }
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < nkv; ++j) {
@@ -225,7 +231,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           tma_load_3d(sV + vs * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_v, vb, c * 64, j * BN, bh);
         ++v_issued;
       }
-      wait_drain(bq, 0, to);
+      if (load_qdo) wait_drain(bq, 0, to);
       for (int x = (k_issued > C::DQ_KS ? k_issued - C::DQ_KS : 0); x < k_issued; ++x)
         wait_drain(smem_u32(&bars->k_full[x % C::DQ_KS]), (x / C::DQ_KS) & 1, to);
       for (int x = (v_issued > C::DQ_VS ? v_issued - C::DQ_VS : 0); x < v_issued; ++x)
@@ -456,10 +462,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   if (warp == BWD_PRODUCER_WARP) {
     if (lane == 0) {
       const uint32_t bkv = smem_u32(&bars->kv_full);
-      mbar_arrive_expect_tx(bkv, 2 * C::TILE_BYTES);
-      for (int c = 0; c < C::KCH; ++c) {
-        tma_load_3d(sK + c * C::CHUNK_BYTES, &tm_k, bkv, c * 64, k0, bh);
-        tma_load_3d(sV + c * C::CHUNK_BYTES, &tm_v, bkv, c * 64, k0, bh);
+      const bool load_kv = p.inject_timeout != 2;
+      if (load_kv) {
+        mbar_arrive_expect_tx(bkv, 2 * C::TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c) {
+          tma_load_3d(sK + c * C::CHUNK_BYTES, &tm_k, bkv, c * 64, k0, bh);
+          tma_load_3d(sV + c * C::CHUNK_BYTES, &tm_v, bkv, c * 64, k0, bh);
+        }
       }
       int issued = 0;
       for (int t = 0; t < nq; ++t) {
@@ -479,7 +488,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         bulk_load_1d(sv + 512, p.dvec + vec_head + i * BM, 512, bq);
         ++issued;
       }
-      wait_drain(bkv, 0, to);
+      if (load_kv) wait_drain(bkv, 0, to);
       for (int x = (issued > C::KV_QS ? issued - C::KV_QS : 0); x < issued; ++x)
         wait_drain(smem_u32(&bars->q_full[x % C::KV_QS]), (x / C::KV_QS) & 1, to);
     }

@@ -42,6 +42,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdint>
@@ -70,7 +71,7 @@ __host__ __device__ constexpr uint32_t tm_s(int t) { return 128u * static_cast<u
 __host__ __device__ constexpr uint32_t tm_o(int t) { return 256u + 128u * static_cast<uint32_t>(t); }
 constexpr float RESCALE_THRESHOLD = 8.0f;
 #ifndef FA2_EMU_PAIRS_D128
-#define FA2_EMU_PAIRS_D128 2
+#define FA2_EMU_PAIRS_D128 1
 #endif
 #ifndef FA2_EMU_PAIRS_D64
 #define FA2_EMU_PAIRS_D64 3
@@ -767,19 +768,19 @@ static int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
                     const Params& prm, int B, int H, cudaStream_t stream) {
   using C = Cfg<HD>;
   auto kern = fa2_fwd_kernel<HD, CAUSAL>;
-  static int attr_done_mask = 0;  // per device bit (devices 0..31)
+  static std::atomic<unsigned> attr_done_mask{0};  // per device bit (devices 0..31)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
     set_detail("cudaGetDevice failed");
     return FA2_ERR_CUDA;
   }
-  if (dev >= 32 || !(attr_done_mask & (1 << dev))) {
+  if (dev >= 32 || !(attr_done_mask.load(std::memory_order_acquire) & (1u << dev))) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) {
       set_detail("cudaFuncSetAttribute: %s", cudaGetErrorString(e));
       return FA2_ERR_CUDA;
     }
-    if (dev < 32) attr_done_mask |= (1 << dev);
+    if (dev < 32) attr_done_mask.fetch_or(1u << dev, std::memory_order_acq_rel);
   }
   dim3 grid(B * H * prm.n_q_blocks);
   kern<<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, prm);
@@ -816,7 +817,7 @@ static int causal_group_heads(int BH, int N, int d, int n_q_blocks) {
 
 static int splitkv_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
                         int Nk, int d, int causal, float scale, int n_splits, void* workspace,
-                        size_t workspace_bytes, cudaStream_t stream);
+                        size_t workspace_bytes, unsigned long long timeout_ns, int inject, cudaStream_t stream);
 
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                     int causal, float scale, unsigned long long timeout_ns, int inject, cudaStream_t stream) {
@@ -826,11 +827,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   if (padded_hd(d) == 256) {
     // d = 256 runs on the one-tile kernel of the split-K/V path (64-key tiles)
     // as a single key range with Nq = Nk, which writes O and LSE directly.
-    if (inject) {
-      set_detail("the timeout test hook covers the 32..128-column kernel only");
-      return FA2_ERR_UNSUPPORTED;
-    }
-    return splitkv_impl(q, k, v, o, lse, B, H, N, N, d, causal, scale, 1, nullptr, 0, stream);
+    return splitkv_impl(q, k, v, o, lse, B, H, N, N, d, causal, scale, 1, nullptr, 0, timeout_ns, inject, stream);
   }
   CUtensorMap tq, tk, tv, to;
   const int BH = B * H;
@@ -903,19 +900,19 @@ static int skv_launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
                         int n_q_tiles, int splits, __nv_bfloat16* o, float* lse, cudaStream_t stream) {
   using C = SkvCfg<HD>;
   auto kern = fa2_splitkv_kernel<HD, CAUSAL, QUAD>;
-  static int attr_done_mask = 0;  // per device bit (devices 0..31)
+  static std::atomic<unsigned> attr_done_mask{0};  // per device bit (devices 0..31)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
     set_detail("cudaGetDevice failed");
     return FA2_ERR_CUDA;
   }
-  if (dev >= 32 || !(attr_done_mask & (1 << dev))) {
+  if (dev >= 32 || !(attr_done_mask.load(std::memory_order_acquire) & (1u << dev))) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) {
       set_detail("cudaFuncSetAttribute: %s", cudaGetErrorString(e));
       return FA2_ERR_CUDA;
     }
-    if (dev < 32) attr_done_mask |= (1 << dev);
+    if (dev < 32) attr_done_mask.fetch_or(1u << dev, std::memory_order_acq_rel);
   }
   kern<<<dim3(n_q_tiles, prm.BH, splits), SKV_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, prm);
   cudaError_t e = cudaGetLastError();
@@ -937,7 +934,7 @@ static int skv_launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
 
 static int splitkv_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
                         int Nk, int d, int causal, float scale, int n_splits, void* workspace,
-                        size_t workspace_bytes, cudaStream_t stream) {
+                        size_t workspace_bytes, unsigned long long timeout_ns, int inject, cudaStream_t stream) {
   g_detail[0] = 0;
   if (!q || !k || !v || !o || !lse) {
     set_detail("null pointer");
@@ -1001,7 +998,8 @@ static int splitkv_impl(const void* q, const void* k, const void* v, void* o, fl
   prm.n_kv_tiles = (Nk + skv_tile_keys(d) - 1) / skv_tile_keys(d);
   prm.tiles_per_split = (prm.n_kv_tiles + splits - 1) / splits;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
-  prm.timeout_ns = DEFAULT_TIMEOUT_NS;
+  prm.timeout_ns = timeout_ns;
+  prm.inject_timeout = inject;
   const int n_q_tiles = (Nq + BM - 1) / BM;
   auto* ob = static_cast<__nv_bfloat16*>(o);
   if (padded_hd(d) == 64) {
@@ -1034,7 +1032,7 @@ template <int HD, bool CAUSAL>
 static int bwd_launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                         const BwdParams& prm, cudaStream_t stream) {
   using C = BwdCfg<HD>;
-  static int attr_done_mask = 0;  // per device bit (devices 0..31)
+  static std::atomic<unsigned> attr_done_mask{0};  // per device bit (devices 0..31)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
     set_detail("cudaGetDevice failed");
@@ -1042,14 +1040,14 @@ static int bwd_launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
   }
   auto kq = fa2_bwd_dq_kernel<HD, CAUSAL>;
   auto kkv = fa2_bwd_dkdv_kernel<HD, CAUSAL>;
-  if (dev >= 32 || !(attr_done_mask & (1 << dev))) {
+  if (dev >= 32 || !(attr_done_mask.load(std::memory_order_acquire) & (1u << dev))) {
     cudaError_t e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::DQ_SMEM);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, C::KV_SMEM);
     if (e != cudaSuccess) {
       set_detail("cudaFuncSetAttribute: %s", cudaGetErrorString(e));
       return FA2_ERR_CUDA;
     }
-    if (dev < 32) attr_done_mask |= (1 << dev);
+    if (dev < 32) attr_done_mask.fetch_or(1u << dev, std::memory_order_acq_rel);
   }
   const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_tiles);
   kq<<<grid, BWD_THREADS, C::DQ_SMEM, stream>>>(tq, tk, tv, tdo, prm);
@@ -1069,7 +1067,8 @@ static int bwd_launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
 
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                     void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
-                    void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+                    void* workspace, size_t workspace_bytes, unsigned long long timeout_ns, int inject,
+                    cudaStream_t stream) {
   g_detail[0] = 0;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) {
     set_detail("null pointer");
@@ -1141,7 +1140,8 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   prm.group_heads = causal ? causal_group_heads(static_cast<int>(BH), N, d, prm.n_tiles) : 1;
   prm.scale = scale;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
-  prm.timeout_ns = DEFAULT_TIMEOUT_NS;
+  prm.timeout_ns = timeout_ns;
+  prm.inject_timeout = inject;
   if (padded_hd(d) == 64)
     return causal ? bwd_launch_t<64, true>(tq, tk, tv, tdo, prm, stream)
                   : bwd_launch_t<64, false>(tq, tk, tv, tdo, prm, stream);
@@ -1351,7 +1351,18 @@ int fa2_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float*
                     int d, int causal, float scale, int n_splits, void* workspace, size_t workspace_bytes,
                     void* stream) {
   return fa2::splitkv_impl(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, n_splits, workspace, workspace_bytes,
-                           static_cast<cudaStream_t>(stream));
+                           fa2::DEFAULT_TIMEOUT_NS, 0, static_cast<cudaStream_t>(stream));
+}
+
+int fa2_fwd_splitkv_inject_timeout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                                   int Nq, int Nk, int d, int causal, float scale, int n_splits, void* workspace,
+                                   size_t workspace_bytes, unsigned long long timeout_ns, void* stream) {
+  if (timeout_ns == 0 || timeout_ns > fa2::DEFAULT_TIMEOUT_NS) {
+    fa2::set_detail("timeout_ns out of range (1 .. 2e9)");
+    return FA2_ERR_INVALID_ARG;
+  }
+  return fa2::splitkv_impl(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, n_splits, workspace, workspace_bytes,
+                           timeout_ns, 1, static_cast<cudaStream_t>(stream));
 }
 
 int fa2_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
@@ -1362,7 +1373,7 @@ int fa2_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o,
     return FA2_ERR_INVALID_ARG;
   }
   size_t need = 0;
-  if (fa2::skv_sizes_ok(B, H, Nq, Nk) && n_splits >= 0 && (d == 64 || d == 128)) {
+  if (fa2::skv_sizes_ok(B, H, Nq, Nk) && n_splits >= 0 && fa2::d_supported(d)) {
     const int splits = fa2::skv_resolve_splits(B, H, Nq, Nk, n_splits, fa2::skv_tile_keys(d));
     need = fa2::skv_workspace_bytes(B, H, Nq, fa2::padded_hd(d), splits);
     if (need > FA2_SPLITKV_STATIC_SCRATCH_BYTES) {
@@ -1379,7 +1390,7 @@ int fa2_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o,
   }
   return fa2::splitkv_impl(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, n_splits, scratch,
                            scratch ? static_cast<size_t>(FA2_SPLITKV_STATIC_SCRATCH_BYTES) : 0,
-                           static_cast<cudaStream_t>(stream));
+                           fa2::DEFAULT_TIMEOUT_NS, 0, static_cast<cudaStream_t>(stream));
 }
 
 size_t fa2_bwd_workspace_bytes(int B, int H, int N, int d) {
@@ -1391,7 +1402,23 @@ int fa2_bwd(const void* q, const void* k, const void* v, const void* o, const vo
             void* dk, void* dv, int B, int H, int N, int d, int causal, float scale, void* workspace,
             size_t workspace_bytes, void* stream) {
   return fa2::bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, workspace, workspace_bytes,
-                       static_cast<cudaStream_t>(stream));
+                       fa2::DEFAULT_TIMEOUT_NS, 0, static_cast<cudaStream_t>(stream));
+}
+
+int fa2_bwd_inject_timeout(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                           const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal,
+                           float scale, void* workspace, size_t workspace_bytes, int kernel,
+                           unsigned long long timeout_ns, void* stream) {
+  if (timeout_ns == 0 || timeout_ns > fa2::DEFAULT_TIMEOUT_NS) {
+    fa2::set_detail("timeout_ns out of range (1 .. 2e9)");
+    return FA2_ERR_INVALID_ARG;
+  }
+  if (kernel != 0 && kernel != 1) {
+    fa2::set_detail("kernel must be 0 (dQ) or 1 (dK/dV)");
+    return FA2_ERR_INVALID_ARG;
+  }
+  return fa2::bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, workspace, workspace_bytes,
+                       timeout_ns, kernel + 1, static_cast<cudaStream_t>(stream));
 }
 
 const char* fa2_strerror(int status) {

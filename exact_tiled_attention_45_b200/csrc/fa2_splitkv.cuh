@@ -80,6 +80,7 @@ struct SkvParams {
   int tiles_per_split;  // key tiles per range
   float scale_log2;
   unsigned long long timeout_ns;
+  int inject_timeout;  // test hook: withhold the query load so the waits on it run out
 };
 
 struct SkvBarriers {
@@ -182,14 +183,18 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
   if (warp == SKV_PRODUCER_WARP) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(b_q, C::Q_BYTES);
-      if constexpr (QUAD) {
-        // Four copies of the (at most 32) query rows, 32-row boxes, at rows
-        // 0, 32, 64, 96 of the tile; rows past Nq are zero-filled.
-        for (int w = 0; w < 4; ++w)
-          for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * C::Q_CHUNK + w * 32 * 128, &tm_q, b_q, c * 64, 0, bh);
-      } else {
-        for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * C::Q_CHUNK, &tm_q, b_q, c * 64, q_first, bh);
+      const bool load_q = !p.inject_timeout;
+      if (load_q) {
+        mbar_arrive_expect_tx(b_q, C::Q_BYTES);
+        if constexpr (QUAD) {
+          // Four copies of the (at most 32) query rows, 32-row boxes, at rows
+          // 0, 32, 64, 96 of the tile; rows past Nq are zero-filled.
+          for (int w = 0; w < 4; ++w)
+            for (int c = 0; c < C::KCH; ++c)
+              tma_load_3d(sQ + c * C::Q_CHUNK + w * 32 * 128, &tm_q, b_q, c * 64, 0, bh);
+        } else {
+          for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * C::Q_CHUNK, &tm_q, b_q, c * 64, q_first, bh);
+        }
       }
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < nkv; ++j) {
@@ -213,7 +218,7 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
           tma_load_3d(sV + vs * C::KV_BYTES + c * C::KV_CHUNK, &tm_v, vb, c * 64, kv0, bh);
         ++v_issued;
       }
-      wait_drain(b_q, 0, to);
+      if (load_q) wait_drain(b_q, 0, to);
       for (int x = (k_issued > C::KS ? k_issued - C::KS : 0); x < k_issued; ++x)
         wait_drain(smem_u32(&bars->k_full[x % C::KS]), (x / C::KS) & 1, to);
       for (int x = (v_issued > C::VS ? v_issued - C::VS : 0); x < v_issued; ++x)

@@ -57,7 +57,6 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
-// 3-D tiled bulk tensor load global -> shared, completion counted on `bar`.
 // Untiled bulk copy global -> shared (no multicast): both addresses 16-byte
 // aligned, size a multiple of 16 bytes; completes bytes on the mbarrier.
 __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
@@ -66,6 +65,7 @@ __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint
                : "memory");
 }
 
+// 3-D tiled bulk tensor load global -> shared, completion counted on `bar`.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar, int x, int y,
                                             int z) {
   asm volatile(

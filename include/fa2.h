@@ -95,13 +95,21 @@ size_t fa2_fwd_host_workspace_bytes(int B, int H, int N, int d);
  * Synchronise `stream`, then read and clear the device status word.  Returns
  * FA2_ERR_TIMEOUT if any kernel launched since the last call gave up a bounded
  * wait, FA2_ERR_CUDA if the synchronisation failed, else FA2_OK.
+ *
+ * The status word is one per device for the whole process, not one per
+ * stream or per call: a time-out in a kernel on any stream of the current
+ * device is reported to whichever caller reads the word first (this call, or
+ * fa2_fwd_host, which calls it), and that read clears it for everyone.  Code
+ * that shares a device between independent users and needs to attribute a
+ * time-out must serialise its calls with their fa2_sync_status reads.
  */
 int fa2_sync_status(void* stream);
 
 /*
  * Test hook for the failure path: launch the attention kernel (same
- * arguments as fa2_fwd, d <= 128) with the query-tile load withheld, so every wait on it
- * runs out after `timeout_ns` nanoseconds.  The kernel then sets the status
+ * arguments as fa2_fwd, every supported d; d = 256 runs the one-tile kernel
+ * of fa2_fwd_splitkv) with the query-tile load withheld, so every wait on it
+ * runs out after `timeout_ns` nanoseconds (1 .. 2e9).  The kernel then sets the status
  * word and exits cleanly (tensor memory released, no copy left in flight);
  * fa2_sync_status returns FA2_ERR_TIMEOUT.  Outputs are unspecified.
  */
@@ -155,6 +163,19 @@ int fa2_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float*
                     int d, int causal, float scale, int n_splits, void* workspace, size_t workspace_bytes,
                     void* stream);
 
+/*
+ * Test hook for the failure path of fa2_fwd_splitkv (same arguments, plus
+ * `timeout_ns`, 1 .. 2e9): the range kernel runs with its query load withheld,
+ * so its waits run out after `timeout_ns` nanoseconds; with two or more key
+ * ranges the merge kernel still runs after it, on the unspecified partials.
+ * Every CTA records the time-out, drains its own copies and MMAs, releases
+ * tensor memory and returns; fa2_sync_status returns FA2_ERR_TIMEOUT.
+ * Outputs are unspecified.  Covers the quarter mode (Nq <= 32) as well.
+ */
+int fa2_fwd_splitkv_inject_timeout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                                   int Nq, int Nk, int d, int causal, float scale, int n_splits, void* workspace,
+                                   size_t workspace_bytes, unsigned long long timeout_ns, void* stream);
+
 /* Key ranges fa2_fwd_splitkv uses for these sizes and request (0 on bad sizes). */
 int fa2_fwd_splitkv_splits(int B, int H, int Nq, int Nk, int d, int n_splits);
 
@@ -199,6 +220,21 @@ int fa2_bwd(const void* q, const void* k, const void* v, const void* o, const vo
 
 /* Workspace bytes fa2_bwd needs for this shape (0 on bad sizes). */
 size_t fa2_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Test hook for the failure path of fa2_bwd (same arguments, plus `kernel`
+ * and `timeout_ns`, 1 .. 2e9).  kernel = 0: the dQ kernel runs with its Q/dO
+ * tile load withheld; kernel = 1: the dK/dV kernel runs with its K/V tile load
+ * withheld.  That kernel's waits run out after `timeout_ns`; it records the
+ * time-out, drains its own copies and MMAs, releases tensor memory and
+ * returns; the other kernel runs normally.  fa2_sync_status returns
+ * FA2_ERR_TIMEOUT.  Gradients are unspecified.  kernel outside {0, 1} ->
+ * FA2_ERR_INVALID_ARG.
+ */
+int fa2_bwd_inject_timeout(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                           const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal,
+                           float scale, void* workspace, size_t workspace_bytes, int kernel,
+                           unsigned long long timeout_ns, void* stream);
 
 /*
  * fa2_fwd_splitkv without a workspace argument, for callers that cannot

@@ -100,6 +100,20 @@ def test_inject_hook_validates_timeout(lib):
     assert rc == binding.FA2_ERR_INVALID_ARG
 
 
+def test_splitkv_and_backward_hooks_validate_on_the_host(lib):
+    p = [FAKE + (i << 32) for i in range(10)]
+    rc = lib.fa2_fwd_splitkv_inject_timeout(*p[:5], 1, 2, 1, 1000, 128, 0, 0.088, 2, p[5], 1 << 30,
+                                            ctypes.c_ulonglong(0), None)
+    assert rc == binding.FA2_ERR_INVALID_ARG and b"timeout" in lib.fa2_last_error_detail()
+    rc = lib.fa2_fwd_splitkv_inject_timeout(*p[:5], 1, 2, 1, 1000, 128, 0, 0.088, 2, p[5], 1 << 30,
+                                            ctypes.c_ulonglong(3_000_000_000), None)
+    assert rc == binding.FA2_ERR_INVALID_ARG
+    for kernel, timeout in ((2, 1000), (-1, 1000), (0, 0)):
+        rc = lib.fa2_bwd_inject_timeout(*p[:9], 1, 2, 200, 128, 0, 0.088, p[9], 1 << 20, kernel,
+                                        ctypes.c_ulonglong(timeout), None)
+        assert rc == binding.FA2_ERR_INVALID_ARG, (kernel, timeout)
+
+
 def test_python_wrapper_rejects_wrong_tensors():
     import torch
     q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
@@ -202,6 +216,18 @@ def test_static_scratch_entry_rejects_on_the_host(lib):
     assert b"static scratch" in lib.fa2_last_error_detail()
     rc = lib.fa2_fwd_splitkv_static(0, FAKE, FAKE, FAKE, FAKE, 1, 1, 1, 128, 64, 0, 0.125, 0, None)
     assert rc == binding.FA2_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("d", [32, 96, 256])
+def test_static_scratch_sizes_every_head_dim(lib, d):
+    # The scratch need is computed for every supported head dimension (the
+    # zero-padded 32 and 96, and 256 with its 64-key tiles), so an oversized
+    # request is refused for the scratch's size, not for a missing workspace.
+    assert lib.fa2_fwd_splitkv_workspace_bytes(1, 16, 4096, 4096, d, 32) > binding.SPLITKV_STATIC_SCRATCH_BYTES
+    rc = lib.fa2_fwd_splitkv_static(FAKE, FAKE + (1 << 32), FAKE + (2 << 32), FAKE + (3 << 32), FAKE + (4 << 32),
+                                    1, 16, 4096, 4096, d, 1, 0.088, 32, None)
+    assert rc == binding.FA2_ERR_INVALID_ARG
+    assert b"static scratch" in lib.fa2_last_error_detail()
 
 
 # ---------------------------------------------------------------- backward
