@@ -16,6 +16,18 @@ value is the FLOPs of all ranks divided by the slowest rank's time.
 ``--impl reference`` times the fp64 CPU oracle on this host's cores instead,
 each step on a bounded sample of heads of the same workload (rank 0 only).
 
+The headline is timed as ``--repeats`` regions of exactly K steps, each
+bracketed by a barrier and a synchronisation; the value is from the median
+region.  On one GPU the line also carries ``grid``: every point of the
+16k-token sweep (N = 512 .. 16384, d = 64 and 128, causal off and on, H =
+2048/d, B = 16384/N, plus Q, K x 4 at d = 128, N >= 4096), each timed with
+CUDA events over at least 10 launches, with its fraction of the measured
+bf16 peak, the median SM clock while it ran, its exponential floor and the
+tensor-pipe utilisation from an ncu capture of the same kernel source
+(``profiles/tensor_pipe.txt``, null when the source has changed since).
+``--profile-grid`` launches every grid point once and nothing else (for that
+ncu capture).
+
 Decode workloads (``--workload decode_...`` / ``chunk_...``: Nq queries at the
 end of an Nk-long sequence) run the split-K/V entry point instead; a step is
 one call (range kernel + merge kernel) and the metric is effective HBM GB/s:
@@ -62,6 +74,14 @@ def parse_args():
     ap.add_argument("--no-gemm", action="store_true", help="skip the library GEMM comparator")
     ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
                     help="bwd: time the backward (dQ, dK, dV) instead of the forward")
+    ap.add_argument("--repeats", type=int, default=15, help="bracketed K-step regions of the headline (median)")
+    ap.add_argument("--region-gap-ms", type=float, default=20.0, help="idle gap before each headline region")
+    ap.add_argument("--no-grid", action="store_true", help="skip the sweep over the 16k-token grid")
+    ap.add_argument("--grid-ms", type=float, default=5.0, help="target length of each grid point's timed regions")
+    ap.add_argument("--sustained-ms", type=float, default=1000.0,
+                    help="length of the sustained run of each d=128, N>=4096 grid point (0: skip)")
+    ap.add_argument("--profile-grid", action="store_true",
+                    help="launch the forward once per grid point and exit (for an ncu capture)")
     return ap.parse_args()
 
 
@@ -95,6 +115,181 @@ def recorded_traffic(workload: str, src_hash: str):
     except OSError:
         pass
     return None
+
+
+def recorded_tensor_pipe(src_hash: str):
+    """Per-workload ncu figures of this exact kernel source:
+    {workload: {"tensor_pipe_pct": elapsed %, "tensor_pipe_active_pct": active %, "traffic": bytes}}."""
+    path = os.path.join(ROOT, "profiles", "tensor_pipe.txt")
+    out = {}
+    try:
+        with open(path) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 5 and not line.startswith("#") and parts[0] == src_hash:
+                    out[parts[1]] = {"tensor_pipe_pct": float(parts[2]), "tensor_pipe_active_pct": float(parts[3]),
+                                     "traffic": float(parts[4])}
+    except OSError:
+        pass
+    return out
+
+
+GRID_TOKENS = 16384
+GRID_HIDDEN = 2048
+
+
+def grid_points():
+    """(name, B, H, N, d, causal, qk_mult) of the 16k-token sweep."""
+    pts = []
+    for d in (64, 128):
+        for causal in (False, True):
+            for N in (512, 1024, 2048, 4096, 8192, 16384):
+                pts.append((f"grid_N{N}_d{d}_{'causal' if causal else 'full'}", GRID_TOKENS // N, GRID_HIDDEN // d,
+                            N, d, causal, 1.0))
+    for causal in (False, True):
+        for N in (4096, 8192, 16384):
+            pts.append((f"grid_N{N}_d128_{'causal' if causal else 'full'}_x4", GRID_TOKENS // N, GRID_HIDDEN // 128,
+                        N, 128, causal, 4.0))
+    return pts
+
+
+class GridInputs:
+    """Device copies of the sweep's inputs, drawn once per head dimension.
+
+    Every grid point of one d holds 16384 x 2048 elements per tensor, and
+    make_qkv(B, H, N, d) draws the same flat sequence for every such shape,
+    so one draw per d (viewed as [B, H, N, d]) gives each point exactly the
+    inputs make_qkv would."""
+
+    def __init__(self, dev):
+        self.dev, self.d, self.qkv, self.x4 = dev, None, None, None
+
+    def get(self, B, H, N, d, qk_mult):
+        import torch
+        from exact_tiled_attention_45_b200.inputs import make_qkv
+        if self.d != d:
+            self.qkv = self.x4 = None
+            torch.cuda.empty_cache()
+            self.qkv = [t.to(self.dev) for t in make_qkv(1, 1, GRID_TOKENS * (GRID_HIDDEN // d), d, seed=0)]
+            self.o = torch.empty_like(self.qkv[0])
+            self.lse = torch.empty(GRID_TOKENS * (GRID_HIDDEN // d), dtype=torch.float32, device=self.dev)
+            self.d = d
+        src = self.qkv
+        if qk_mult != 1.0:
+            if self.x4 is None:
+                self.x4 = [self.qkv[0] * 4, self.qkv[1] * 4]
+            src = [self.x4[0], self.x4[1], self.qkv[2]]
+        shp = (B, H, N, d)
+        return [t.view(shp) for t in src], self.o.view(shp), self.lse.view(B, H, N)
+
+
+def run_grid(dev, stream, sampler, peaks, target_ms: float, src: str, sustained_ms: float = 1000.0):
+    """Time every sweep point; returns the ``grid`` object of the bench line.
+
+    Burst timing, like the headline: after a short idle gap, 5 regions of at
+    least 10 back-to-back launches (and at least ``target_ms``), median.  For
+    the d = 128, N >= 4096 points also a sustained run of ``sustained_ms``
+    of back-to-back launches, against the measured sustained bf16 peak (the
+    1 kW power cap lowers the SM clock under long full load)."""
+    import torch
+    import exact_tiled_attention_45_b200 as fa2
+    from exact_tiled_attention_45_b200.inputs import Workload
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    rec = recorded_tensor_pipe(src)
+    inputs = GridInputs(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    points = {}
+    for name, B, H, N, d, causal, mult in grid_points():
+        w = Workload(name, B, H, N, d, causal, mult)
+        (q, k, v), o, lse = inputs.get(B, H, N, d, mult)
+
+        def call():
+            fa2.fwd(q, k, v, causal=causal, out=o, lse=lse, stream=stream)
+
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        call()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        est = max(ev0.elapsed_time(ev1), 1e-3)
+        reps = max(10, int(math.ceil(target_ms / est)))
+        time.sleep(0.25)
+        region_ms, t_start = [], time.time()
+        for _ in range(5):
+            ev0.record(stream)
+            for _ in range(reps):
+                call()
+            ev1.record(stream)
+            torch.cuda.synchronize(dev)
+            region_ms.append(ev0.elapsed_time(ev1) / reps)
+        t_end = time.time()
+        ms = sorted(region_ms)[2]
+        mhz = sampler.median_between(t_start, t_end)
+        sustained = None
+        if sustained_ms > 0 and d == 128 and N >= 4096 and mult == 1.0:
+            n_sus = max(10, int(math.ceil(sustained_ms / est)))
+            ts0 = time.time()
+            ev0.record(stream)
+            for _ in range(n_sus):
+                call()
+            ev1.record(stream)
+            torch.cuda.synchronize(dev)
+            sus_ms = ev0.elapsed_time(ev1) / n_sus
+            sus_tf = w.flops / (sus_ms * 1e-3) / 1e12
+            peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+            sustained = {"ms": round(sus_ms, 5), "tflops": round(sus_tf, 1), "launches": n_sus,
+                         "seconds": round(time.time() - ts0, 2),
+                         "sm_mhz": sampler.median_between(ts0, time.time()),
+                         "frac_of_sustained_peak": round(sus_tf / peak_sus, 4),
+                         "frac_of_burst_peak": round(sus_tf / peak, 4)}
+        sm_hz = float(mhz or peaks.get("sm_max_mhz", 1965.0)) * 1e6
+        tflops = w.flops / (ms * 1e-3) / 1e12
+        r = rec.get(name, {})
+        points[name] = {
+            "B": B, "H": H, "N": N, "d": d, "causal": causal, "qk_mult": mult,
+            "ms": round(ms, 5), "tflops": round(tflops, 1), "frac": round(tflops / peak, 4),
+            "launches": 5 * reps, "sm_mhz": mhz, "sustained": sustained,
+            "exp_bound_pct": round(100.0 * w.exps / (EX2_PER_CLK_PER_SM * sms * sm_hz) / (ms * 1e-3), 1),
+            "tensor_pipe_pct": r.get("tensor_pipe_pct"), "tensor_pipe_active_pct": r.get("tensor_pipe_active_pct"),
+            "traffic": r.get("traffic"), "algorithmic_bytes": w.io_bytes,
+        }
+    fa2.sync_status(stream)
+    del inputs
+    torch.cuda.empty_cache()
+    target = [p for n, p in points.items() if p["d"] == 128 and p["N"] >= 4096 and p["qk_mult"] == 1.0]
+    return {
+        "points": points,
+        "timing": ("burst: after a 250 ms idle gap, median of 5 CUDA-event regions of >= 10 back-to-back launches "
+                   "(>= grid-ms each; inputs 201 MB > L2); sustained (d=128, N>=4096): one region of "
+                   "back-to-back launches for sustained-ms"),
+        "peak": peak, "peak_source": "measured bf16 burst",
+        "tensor_pipe_source": "ncu sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_elapsed, one launch per "
+                              "point, profiles/tensor_pipe.txt (null unless captured on this kernel source)",
+        "d128_N_ge_4k": {"min_frac": min(p["frac"] for p in target), "max_frac": max(p["frac"] for p in target),
+                          "target_frac": 0.60, "met": all(p["frac"] >= 0.60 for p in target),
+                          "sustained_min_frac_of_sustained_peak": min(
+                              (p["sustained"]["frac_of_sustained_peak"] for p in target if p["sustained"]),
+                              default=None)},
+    }
+
+
+def profile_grid():
+    """One forward launch per grid point, nothing else (the ncu capture)."""
+    import torch
+    import exact_tiled_attention_45_b200 as fa2
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    inputs = GridInputs(dev)
+    for name, B, H, N, d, causal, mult in grid_points():
+        (q, k, v), o, lse = inputs.get(B, H, N, d, mult)
+        fa2.fwd(q, k, v, causal=causal, out=o, lse=lse, stream=stream)
+        fa2.sync_status(stream)
+        print(name, flush=True)
+    return 0
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -134,7 +329,7 @@ class ClockSampler:
     }
 
     def __init__(self, torch_device):
-        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self.samples, self.stamps, self.reasons, self.max_mhz = [], [], 0, None
         self._stop = threading.Event()
         self._thread = None
         try:
@@ -155,9 +350,15 @@ class ClockSampler:
         nv = self._nv
         try:
             self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+            self.stamps.append(time.time())
             self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
         except Exception:
             pass
+
+    def median_between(self, t0: float, t1: float):
+        """Median SM clock of the samples taken between two wall-clock times."""
+        s = sorted(m for m, t in zip(list(self.samples), list(self.stamps)) if t0 <= t <= t1)
+        return s[len(s) // 2] if s else None
 
     def _run(self):
         while not self._stop.is_set():
@@ -175,10 +376,17 @@ class ClockSampler:
             self._thread.join()
             self._sample()
 
-    def summary(self):
+    def summary(self, windows=None):
+        """Median SM clock and throttle reasons; with `windows` (pairs of wall
+        times) only the samples taken inside them count for the median."""
         if self._nv is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
         s = sorted(self.samples)
+        if windows:
+            inside = sorted(m for m, t in zip(list(self.samples), list(self.stamps))
+                            if any(a <= t <= b for a, b in windows))
+            if inside:
+                s = inside
         med = s[len(s) // 2] if s else None
         names = [k for k, bit in self.REASONS.items() if self.reasons & bit and k != "gpu_idle"]
         return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(s)}
@@ -622,8 +830,10 @@ def main():
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
-    if args.steps < 1 or args.warmup < 3:
-        raise SystemExit("need --steps >= 1 and --warmup >= 3")
+    if args.profile_grid:
+        return profile_grid()
+    if args.steps < 1 or args.warmup < 3 or args.repeats < 1:
+        raise SystemExit("need --steps >= 1, --warmup >= 3 and --repeats >= 1")
     if is_decode(w):
         return run_decode(args, w)
     if args.pass_ == "bwd":
@@ -671,32 +881,42 @@ def main():
 
     sampler = ClockSampler(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize(dev)
     sampler.start()
-    if flush is None:
-        ev0.record(stream)
-        for _ in range(args.steps):
-            step()
-        ev1.record(stream)
+    # `repeats` regions of exactly K steps, each bracketed by a barrier and a
+    # synchronisation on both sides; the value comes from the median region.
+    # A short idle gap before each region makes every region one burst of K
+    # steps (back-to-back regions would add up to a sustained load, which the
+    # power cap throttles; the sweep below reports sustained figures too).
+    region_ms, windows = [], []
+    for _ in range(args.repeats):
+        time.sleep(args.region_gap_ms * 1e-3)
+        barrier()
         torch.cuda.synchronize(dev)
-        total_ms = ev0.elapsed_time(ev1)
-        kernel_ms = total_ms / args.steps
-    else:
-        # L2 is flushed before every step; only the kernels are timed.
-        kernel_ms_sum = 0.0
-        for _ in range(args.steps):
-            flush.zero_()
+        t_win = time.time()
+        if flush is None:
             ev0.record(stream)
-            fa2.fwd(q, k, v, causal=w.causal, out=o, lse=lse, stream=stream)
+            for _ in range(args.steps):
+                step()
             ev1.record(stream)
-            ev1.synchronize()
-            kernel_ms_sum += ev0.elapsed_time(ev1)
-        total_ms = kernel_ms_sum
-        kernel_ms = kernel_ms_sum / args.steps
+            torch.cuda.synchronize(dev)
+            region_ms.append(ev0.elapsed_time(ev1))
+        else:
+            # L2 is flushed before every step; only the kernels are timed.
+            t = 0.0
+            for _ in range(args.steps):
+                flush.zero_()
+                ev0.record(stream)
+                fa2.fwd(q, k, v, causal=w.causal, out=o, lse=lse, stream=stream)
+                ev1.record(stream)
+                ev1.synchronize()
+                t += ev0.elapsed_time(ev1)
+            region_ms.append(t)
+        windows.append((t_win, time.time()))
+        barrier()
     sampler.stop()
-    barrier()
     fa2.sync_status(stream)
+    total_ms = sorted(region_ms)[len(region_ms) // 2]
+    kernel_ms = total_ms / args.steps
 
     max_ms = max_over_ranks(total_ms, dev)
     ms_per_step = max_ms / args.steps
@@ -740,23 +960,34 @@ def main():
                "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes, "steps": e2e_steps}
         del qp, kp, vp, op, lp, ws
 
+    peaks, peak_kind = load_peaks()
+    src = source_hash()
+    grid = None
+    if not args.no_grid and world == 1:
+        del q, k, v, o, lse
+        torch.cuda.empty_cache()
+        gsampler = ClockSampler(dev)
+        gsampler.start()
+        grid = run_grid(dev, stream, gsampler, peaks, args.grid_ms, src, args.sustained_ms)
+        gsampler.stop()
+        grid["clocks"] = gsampler.summary()
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return 0
 
-    peaks, peak_kind = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     achieved = w.flops / (kernel_ms * 1e-3) / 1e12
-    src = source_hash()
     traffic = recorded_traffic(w.name, src)
 
     def pct(p):
         return step_times[min(len(step_times) - 1, int(round(p / 100.0 * (len(step_times) - 1))))]
 
-    clocks = sampler.summary()
+    clocks = sampler.summary(windows)
+    clocks["basis"] = "samples inside the timed regions"
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     sm_hz = float(clocks.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)) * 1e6
@@ -787,15 +1018,18 @@ def main():
                         "spec_2250": 100.0 * achieved / SPEC_BF16_TFLOPS, "peaks": peak_kind},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_kind} bf16 burst",
-                     "kernel": "fa2_fwd_kernel", "src": src},
+                     "kernel": "fa2_fwd_kernel", "src": src,
+                     "tensor_pipe_pct": recorded_tensor_pipe(src).get(w.name, {}).get("tensor_pipe_pct")},
         "step_ms": {"median": pct(50), "p10": pct(10), "p90": pct(90), "n": len(step_times),
                     "pass": "second pass, one event pair per launch"},
+        "regions_ms": [round(x, 4) for x in region_ms], "repeats": args.repeats,
         "floors": floors,
         "clocks": clocks,
         "gpu_launches": args.steps,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "gemm_comparator": gemm,
+        "grid": grid,
     }
     print(json.dumps(line), flush=True)
     return 0
