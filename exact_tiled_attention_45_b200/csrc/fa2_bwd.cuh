@@ -19,7 +19,7 @@
 // the other operand's tiles, with P and dS recomputed per tile pair:
 //   fa2_bwd_dq_kernel    one CTA per query tile: S = Q K_j^T, dP = dO V_j^T,
 //                        dQ += dS K_j (3 MMAs per key tile); it also writes
-//                        lse2 = LSE * log2(e) and D per row to the workspace;
+//                        -LSE * log2(e) and D per row to the workspace;
 //   fa2_bwd_dkdv_kernel  one CTA per key tile: S^T = K Q_i^T, dP^T = V dO_i^T,
 //                        dV += P^T dO_i, dK += dS^T Q_i (4 MMAs per query tile).
 // Seven MMAs per tile pair instead of five: dQ is not accumulated across CTAs.
@@ -33,6 +33,42 @@ constexpr int BWD_THREADS = 192;
 constexpr int BWD_PRODUCER_WARP = 4;
 constexpr int BWD_MMA_WARP = 5;
 constexpr float LOG2E_F = 1.4426950408889634f;
+// Of every 8 pairs of exponentials 2^(c*s - LSE*log2(e)), this many run on
+// the FMA-pipe polynomial (exp2_poly_pair) and the rest on the
+// special-function unit; the arguments are <= 0 (P <= 1), -inf when masked.
+#ifndef FA2_BWD_EMU_PAIRS
+#define FA2_BWD_EMU_PAIRS 2
+#endif
+
+// P of 128 keys (or queries) of one row: pr[e] = 2^(c * s[e] + nl[e]), where
+// nl is -LSE*log2(e) (one value per row, or per column when `per_col`);
+// masked entries (e past `lim` on a masked tile, see the callers) give 0.
+template <bool PER_COL>
+__device__ __forceinline__ void bwd_probs(float (&pr)[128], const uint32_t (&s)[128], float c, float nl_row,
+                                          const float* nl_col, bool masked, int lim, bool mask_below) {
+  const uint64_t cc = f2_pack(c, c);
+  const uint64_t nlr = f2_pack(nl_row, nl_row);
+#pragma unroll
+  for (int e = 0; e < 128; e += 2) {
+    float x0 = __uint_as_float(s[e]), x1 = __uint_as_float(s[e + 1]);
+    if (masked) {
+      // mask_below: entries before `lim` are masked, else entries after it
+      if (mask_below ? (e < lim) : (e > lim)) x0 = -INFINITY;
+      if (mask_below ? (e + 1 < lim) : (e + 1 > lim)) x1 = -INFINITY;
+    }
+    uint64_t nl = nlr;
+    if (PER_COL) nl = *reinterpret_cast<const uint64_t*>(nl_col + e);
+    const uint64_t x = f2_fma(f2_pack(x0, x1), cc, nl);
+    if (((e >> 1) & 7) < FA2_BWD_EMU_PAIRS) {
+      f2_unpack(exp2_poly_pair(x), pr[e], pr[e + 1]);
+    } else {
+      float a0, a1;
+      f2_unpack(x, a0, a1);
+      pr[e] = ex2(a0);
+      pr[e + 1] = ex2(a1);
+    }
+  }
+}
 
 template <int HD>
 struct BwdCfg {
@@ -64,7 +100,7 @@ struct BwdParams {
   const __nv_bfloat16* o;     // forward output [B*H, N, d]
   const __nv_bfloat16* dout;  // upstream gradient [B*H, N, d]
   const float* lse;           // forward logsumexp (natural log) [B*H, N]
-  float* lse2;                // workspace [B*H, n_tiles*128]: LSE * log2(e); +inf past N
+  float* lse2;                // workspace [B*H, n_tiles*128]: -LSE * log2(e); -inf past N
   float* dvec;                // workspace [B*H, n_tiles*128]: D; 0 past N
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
@@ -304,9 +340,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const int row = q0 + r;
     const bool valid = row < p.N;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    // D = dO . O and lse2 of this row, kept in registers and written to the
-    // workspace for the dK/dV kernel (padding rows: D = 0, lse2 = +inf).
-    float dsum = 0.f, lse2 = INFINITY;
+    // D = dO . O and -LSE*log2(e) of this row, kept in registers and written
+    // to the workspace for the dK/dV kernel (padding rows: D = 0, -inf).
+    float dsum = 0.f, nlse2 = -INFINITY;
     if (valid) {
       const size_t off = (static_cast<size_t>(bh) * p.N + row) * p.d;
       const uint4* o4 = reinterpret_cast<const uint4*>(p.o + off);
@@ -321,11 +357,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           dsum = fmaf(__uint_as_float(aw[e] & 0xffff0000u), __uint_as_float(gw[e] & 0xffff0000u), dsum);
         }
       }
-      lse2 = p.lse[static_cast<size_t>(bh) * p.N + row] * LOG2E_F;
+      nlse2 = -p.lse[static_cast<size_t>(bh) * p.N + row] * LOG2E_F;
     }
     const size_t vrow = static_cast<size_t>(bh) * p.n_tiles * BM + q0 + r;
     p.dvec[vrow] = dsum;
-    p.lse2[vrow] = lse2;
+    p.lse2[vrow] = nlse2;
 
     const float c = p.scale_log2;
     bool ok = true;
@@ -349,11 +385,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         const bool diag = CAUSAL && (j == qt);  // key column e visible iff e <= r
         const bool tail = !CAUSAL && (kv0 + BN > p.N);
         const int lim = diag ? r : (p.N - 1 - kv0);  // last allowed key column
-#pragma unroll
-        for (int e = 0; e < 128; ++e) {
-          const float x = (diag || tail) && e > lim ? -INFINITY : __uint_as_float(s[e]);
-          pr[e] = ex2(x * c - lse2);
-        }
+        bwd_probs<false>(pr, s, c, nlse2, nullptr, diag || tail, lim, false);
       }
       ok = wait_warp(smem_u32(&bars->dp_full), j & 1, abort_flag, to);
       if (!ok) break;
@@ -564,7 +596,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
            wait_warp(smem_u32(&bars->q_full[s]), (t / C::KV_QS) & 1, abort_flag, to);
       if (!ok) break;
       tc_fence_after();
-      const float* l2 = vec + s * 256;  // lse2 of the tile's 128 queries (+inf past N)
+      const float* l2 = vec + s * 256;  // -LSE*log2(e) of the tile's 128 queries (-inf past N)
       const float* dd = l2 + 128;       // D of the tile's 128 queries
       float pr[128];
       {
@@ -576,11 +608,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
         const bool diag = CAUSAL && (i == kt);  // query 128i + e sees this key only if e >= r
-#pragma unroll
-        for (int e = 0; e < 128; ++e) {
-          const float x = (diag && e < r) ? -INFINITY : __uint_as_float(sv[e]);
-          pr[e] = ex2(x * c - l2[e]);
-        }
+        bwd_probs<true>(pr, sv, c, 0.f, l2, diag, r, true);
       }
       // P^T (bf16) over the first 64 score columns, for dV += P^T dO.
 #pragma unroll

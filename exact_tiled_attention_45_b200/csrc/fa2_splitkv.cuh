@@ -20,8 +20,10 @@
 // Partial kernel: one CTA per (128-row query tile, batch*head, key range);
 // 192 threads: warps 0-3 softmax (thread r <-> row r <-> TMEM lane r), warp 4
 // TMA producer, warp 5 MMA issuer.  TMEM: two score buffers (the next S is
-// computed while the softmax works on the current one), a separate P buffer,
-// and O.  Rows past Nq are computed on zero queries and never stored.
+// computed while the softmax works on the current one), two P buffers (the
+// softmax writes P(j+1) while P V(j) still reads P(j); it waits for P V(j)
+// only to rescale O), and O.  Rows past Nq are computed on zero queries and
+// never stored.
 //
 // Quarter mode (QUAD, at most 32 query rows, d <= 128): the query rows are
 // loaded four times, into TMEM lane quadrants 0, 32, 64 and 96, so every
@@ -61,9 +63,10 @@ struct SkvCfg {
   static constexpr int OFF_BAR = OFF_V + VS * KV_BYTES;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  // TMEM columns: S0, S1 (SBN each), P (SBN/2 packed bf16 pairs), O (HD).
+  // TMEM columns: S0, S1 (SBN each), P0, P1 (SBN/2 packed bf16 pairs each), O (HD).
   static constexpr uint32_t TM_S0 = 0, TM_S1 = SBN, TM_P = 2 * SBN, TM_O = (HD == 256) ? 256 : 384;
-  static_assert(TM_P + SBN / 2 <= TM_O && TM_O + HD <= 512, "TMEM budget");
+  __host__ __device__ static constexpr uint32_t tm_p(int b) { return TM_P + static_cast<uint32_t>(b) * (SBN / 2); }
+  static_assert(TM_P + SBN <= TM_O && TM_O + HD <= 512, "TMEM budget");
 };
 
 struct SkvParams {
@@ -88,8 +91,8 @@ struct SkvBarriers {
   uint64_t k_full[4], k_empty[4];
   uint64_t v_full[4], v_empty[4];
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full;
-  uint64_t pv_done;
+  uint64_t p_full[2];   // P buffer b written (by all four softmax warps)
+  uint64_t pv_done[2];  // the P V MMA reading P buffer b complete
   uint64_t mma_final;
   uint32_t tmem_base;
   int abort;
@@ -141,8 +144,6 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
   const uint32_t sK = base + C::OFF_K;
   const uint32_t sV = base + C::OFF_V;
   const uint32_t b_q = smem_u32(&bars->q_full);
-  const uint32_t b_p = smem_u32(&bars->p_full);
-  const uint32_t b_pv = smem_u32(&bars->pv_done);
   const uint32_t b_final = smem_u32(&bars->mma_final);
 
   if (threadIdx.x == 0) {
@@ -159,8 +160,10 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
       mbar_init(smem_u32(&bars->s_full[s]), 1);
       mbar_init(smem_u32(&bars->s_free[s]), 4);
     }
-    mbar_init(b_p, 4);
-    mbar_init(b_pv, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&bars->p_full[b]), 4);
+      mbar_init(smem_u32(&bars->pv_done[b]), 1);
+    }
     mbar_init(b_final, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -254,16 +257,17 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
         if (j >= 1) {
           const int i = j - 1;
           const int vs = i % C::VS;
-          if (!wait_bounded(b_p, i & 1, abort_flag, to, ROLE_MMA)) break;
+          const int pb = i & 1;
+          if (!wait_bounded(smem_u32(&bars->p_full[pb]), (i >> 1) & 1, abort_flag, to, ROLE_MMA)) break;
           if (!wait_bounded(smem_u32(&bars->v_full[vs]), (i / C::VS) & 1, abort_flag, to, ROLE_MMA)) break;
           tc_fence_after();
           const uint32_t vbase = sV + vs * C::KV_BYTES;
 #pragma unroll
           for (int kk = 0; kk < C::SBN / 16; ++kk)
-            mma_ts(tmem + C::TM_O, tmem + C::TM_P + kk * 8,
+            mma_ts(tmem + C::TM_O, tmem + C::tm_p(pb) + kk * 8,
                    smem_desc_sw128(vbase + kk * 2048, C::KV_CHUNK, 1024), IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
           mma_commit(smem_u32(&bars->v_empty[vs]));
-          mma_commit(b_pv);
+          mma_commit(smem_u32(&bars->pv_done[pb]));
         }
       }
       mma_commit(b_final);
@@ -282,8 +286,10 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
       uint32_t z[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) z[e] = 0u;
-      tmem_st32(lane_addr + C::TM_P, z);
-      tmem_st32(lane_addr + C::TM_P + 32, z);
+      tmem_st32(lane_addr + C::tm_p(0), z);
+      tmem_st32(lane_addr + C::tm_p(0) + 32, z);
+      tmem_st32(lane_addr + C::tm_p(1), z);
+      tmem_st32(lane_addr + C::tm_p(1) + 32, z);
       tmem_wait_st();
     }
     float m = -INFINITY, l = 0.f;
@@ -339,12 +345,19 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
       f2_unpack(f2_add(acc[0], acc[1]), r0, r1);
       f2_unpack(f2_add(acc[2], acc[3]), r2, r3);
       const float rowsum = (r0 + r1) + (r2 + r3);
-      if (i > 0) {
-        // O and the P buffer are in use by PV(i-1) until it completes.
-        ok = wait_warp(b_pv, (i - 1) & 1, abort_flag, to);
+      const int pb = i & 1;
+      // P buffer pb was last read by PV(i-2); O is accumulated by PV(i-1),
+      // which must be complete only when O is rescaled here.
+      if (i >= 2) {
+        ok = wait_warp(smem_u32(&bars->pv_done[pb]), ((i - 2) >> 1) & 1, abort_flag, to);
         if (!ok) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
+      }
+      if (i > 0 && __any_sync(0xffffffffu, rescale)) {
+        ok = wait_warp(smem_u32(&bars->pv_done[pb ^ 1]), ((i - 1) >> 1) & 1, abort_flag, to);
+        if (!ok) break;
+        tc_fence_after();
+        {
           const uint64_t aa = f2_pack(alpha, alpha);
 #pragma unroll
           for (int c = 0; c < HD / 32; ++c) {
@@ -363,15 +376,15 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
           }
         }
       }
-      tmem_st16(lane_addr + C::TM_P + 16 * warp, pk);
+      tmem_st16(lane_addr + C::tm_p(pb) + 16 * warp, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(b_p);
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[pb]));
       l = l * alpha + rowsum;
       m = m_new;
     }
-    if (ok) ok = wait_warp(b_pv, (nkv - 1) & 1, abort_flag, to);
+    if (ok) ok = wait_warp(smem_u32(&bars->pv_done[(nkv - 1) & 1]), ((nkv - 1) >> 1) & 1, abort_flag, to);
     // Merge of the four quarters.  Every softmax warp reaches both named
     // barriers whatever happened above (after a time-out the values are
     // unspecified, as documented, but no warp is left waiting).  The K ring
@@ -535,12 +548,19 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[sb]));
       }
-      if (i > 0) {
-        // O and the P buffer are in use by PV(i-1) until it completes.
-        ok = wait_warp(b_pv, (i - 1) & 1, abort_flag, to);
+      const int pb = i & 1;
+      // P buffer pb was last read by PV(i-2); O is accumulated by PV(i-1),
+      // which must be complete only when O is rescaled here.
+      if (i >= 2) {
+        ok = wait_warp(smem_u32(&bars->pv_done[pb]), ((i - 2) >> 1) & 1, abort_flag, to);
         if (!ok) break;
         tc_fence_after();
-        if (live && __any_sync(0xffffffffu, rescale)) {
+      }
+      if (i > 0 && live && __any_sync(0xffffffffu, rescale)) {
+        ok = wait_warp(smem_u32(&bars->pv_done[pb ^ 1]), ((i - 1) >> 1) & 1, abort_flag, to);
+        if (!ok) break;
+        tc_fence_after();
+        {
           const uint64_t aa = f2_pack(alpha, alpha);
 #pragma unroll
           for (int c = 0; c < HD / 32; ++c) {
@@ -561,16 +581,16 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
       }
       if (live) {
 #pragma unroll
-        for (int h = 0; h < SBN / 64; ++h) tmem_st32(lane_addr + C::TM_P + 32 * h, pk[h]);
+        for (int h = 0; h < SBN / 64; ++h) tmem_st32(lane_addr + C::tm_p(pb) + 32 * h, pk[h]);
         tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(b_p);
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[pb]));
       l = l * alpha + rowsum;
       m = m_new;
     }
-    if (ok) ok = wait_warp(b_pv, (nkv - 1) & 1, abort_flag, to);
+    if (ok) ok = wait_warp(smem_u32(&bars->pv_done[(nkv - 1) & 1]), ((nkv - 1) >> 1) & 1, abort_flag, to);
     if (ok && live) {
       tc_fence_after();
       const bool store = row < p.Nq;

@@ -207,7 +207,7 @@ size_t fa2_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int 
  *             (256 -> FA2_ERR_UNSUPPORTED); scale > 0.
  *   workspace, workspace_bytes : caller-owned device buffer, 256-byte
  *             aligned, of at least fa2_bwd_workspace_bytes(B,H,N,d) bytes;
- *             it carries per-row LSE*log2(e) and rowsum(dO o O) from the
+ *             it carries per-row -LSE*log2(e) and rowsum(dO o O) from the
  *             first kernel to the second.  Concurrent calls need separate
  *             workspaces.
  *   stream  : cudaStream_t as void*; two kernels are queued on it.
