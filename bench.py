@@ -533,9 +533,10 @@ def gemm_comparator(w, dev, reps: int = 20) -> dict:
 
 
 def run_backward(args, w):
-    """The backward (fa2_bwd, two kernels) on the workload; TFLOP/s by the
-    usual convention of 2.5 x the forward FLOP (five matmuls; the kernels
-    execute seven, since dQ is computed without atomics)."""
+    """The backward (fa2_bwd: two kernels, three at d = 256) on the workload;
+    TFLOP/s by the usual convention of 2.5 x the forward FLOP (five matmuls;
+    the kernels execute seven, eight at d = 256, since dQ is computed without
+    atomics)."""
     import torch
     import torch.distributed as dist
     import exact_tiled_attention_45_b200 as fa2
@@ -659,7 +660,8 @@ def run_backward(args, w):
         "config": dict(w.as_dict(), seed="rank", scale=f"1/sqrt({w.d})", pass_="bwd",
                        l2=("inputs larger than L2" if flush is None else "L2 flushed before every step"),
                        parallelism=("single GPU" if world == 1 else f"{world} ranks, independent heads, no collective")),
-        "executed_tflops": 3.5 * w.flops / (step_ms * 1e-3) / 1e12,
+        # MMAs per tile pair: 7 (S and dP in both kernels), 8 at d = 256 (S^T in both dK/dV passes)
+        "executed_tflops": (4.0 if w.d > 128 else 3.5) * w.flops / (step_ms * 1e-3) / 1e12,
         "pct_of_peak": {"measured_burst": 100.0 * achieved / peak, "peaks": peak_kind},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": recorded_traffic(w.name + ":bwd", source_hash()),

@@ -26,8 +26,15 @@
 //
 // Roles (192 threads): warps 0-3 elementwise (thread r <-> tile row r <->
 // TMEM lane r), warp 4 TMA producer, warp 5 MMA issuer.  P (dK/dV kernel) and
-// dS are packed to bf16 over the first 64 columns of their score tile in
+// dS are packed to bf16 over the first half of their score tile's columns in
 // TMEM and read from there by the next MMA.  Every wait is bounded.
+//
+// Head dimension 256: the dQ kernel streams 64-key tiles (TMEM: S 64, dP 64
+// and a 256-column dQ; shared memory: Q and dO 128 KB, two K stages, one V
+// stage), and the dK/dV kernel runs twice over 64-query tiles, once for dV
+// (S^T, dV += P^T dO: 320 TMEM columns) and once for dK (S^T, dP^T,
+// dK += dS^T Q: 384 columns), since S^T, dP^T, dV and dK together would need
+// 768 of the 512 columns.  Eight MMAs per tile pair.
 
 constexpr int BWD_THREADS = 192;
 constexpr int BWD_PRODUCER_WARP = 4;
@@ -40,16 +47,16 @@ constexpr float LOG2E_F = 1.4426950408889634f;
 #define FA2_BWD_EMU_PAIRS 2
 #endif
 
-// P of 128 keys (or queries) of one row: pr[e] = 2^(c * s[e] + nl[e]), where
+// P of NC keys (or queries) of one row: pr[e] = 2^(c * s[e] + nl[e]), where
 // nl is -LSE*log2(e) (one value per row, or per column when `per_col`);
 // masked entries (e past `lim` on a masked tile, see the callers) give 0.
-template <bool PER_COL>
-__device__ __forceinline__ void bwd_probs(float (&pr)[128], const uint32_t (&s)[128], float c, float nl_row,
+template <bool PER_COL, int NC>
+__device__ __forceinline__ void bwd_probs(float (&pr)[NC], const uint32_t (&s)[NC], float c, float nl_row,
                                           const float* nl_col, bool masked, int lim, bool mask_below) {
   const uint64_t cc = f2_pack(c, c);
   const uint64_t nlr = f2_pack(nl_row, nl_row);
 #pragma unroll
-  for (int e = 0; e < 128; e += 2) {
+  for (int e = 0; e < NC; e += 2) {
     float x0 = __uint_as_float(s[e]), x1 = __uint_as_float(s[e + 1]);
     if (masked) {
       // mask_below: entries before `lim` are masked, else entries after it
@@ -72,29 +79,42 @@ __device__ __forceinline__ void bwd_probs(float (&pr)[128], const uint32_t (&s)[
 
 template <int HD>
 struct BwdCfg {
+  static_assert(HD == 64 || HD == 128 || HD == 256, "head dimension");
   static constexpr int KCH = HD / 64;
-  static constexpr int CHUNK_BYTES = 128 * 128;
-  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;
-  // dQ kernel: Q and dO resident, K and V rings.
-  static constexpr int DQ_KS = (HD == 128) ? 3 : 4;
-  static constexpr int DQ_VS = (HD == 128) ? 2 : 4;
+  static constexpr int CHUNK_BYTES = 128 * 128;          // 128 rows x 128 bytes
+  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;   // one 128-row tile
+  // dQ kernel: Q and dO resident, K and V rings of BNK-key tiles.
+  static constexpr int BNK = (HD == 256) ? 64 : 128;
+  static constexpr int KV_CHUNK = BNK * 128;
+  static constexpr int KV_TILE = KCH * KV_CHUNK;
+  static constexpr int DQ_KS = (HD == 256) ? 2 : (HD == 128 ? 3 : 4);
+  static constexpr int DQ_VS = (HD == 256) ? 1 : (HD == 128 ? 2 : 4);
   static constexpr int DQ_OFF_Q = 0;
   static constexpr int DQ_OFF_DO = DQ_OFF_Q + TILE_BYTES;
   static constexpr int DQ_OFF_K = DQ_OFF_DO + TILE_BYTES;
-  static constexpr int DQ_OFF_V = DQ_OFF_K + DQ_KS * TILE_BYTES;
-  static constexpr int DQ_OFF_BAR = DQ_OFF_V + DQ_VS * TILE_BYTES;
+  static constexpr int DQ_OFF_V = DQ_OFF_K + DQ_KS * KV_TILE;
+  static constexpr int DQ_OFF_BAR = DQ_OFF_V + DQ_VS * KV_TILE;
   static constexpr int DQ_SMEM = DQ_OFF_BAR + 256 + 1024;
-  // dK/dV kernel: K and V resident, a ring of (Q_i, dO_i, lse2_i, D_i).
-  static constexpr int KV_QS = (HD == 128) ? 2 : 3;
+  // dK/dV kernel: K and V resident (128 keys), a ring of (Q_i, dO_i, lse2_i,
+  // D_i) of BMQ-query tiles.
+  static constexpr int BMQ = (HD == 256) ? 64 : 128;
+  static constexpr int Q_CHUNK = BMQ * 128;
+  static constexpr int Q_TILE = KCH * Q_CHUNK;
+  static constexpr int KV_QS = (HD == 256) ? 1 : (HD == 128 ? 2 : 3);
   static constexpr int KV_OFF_K = 0;
   static constexpr int KV_OFF_V = TILE_BYTES;
   static constexpr int KV_OFF_Q = 2 * TILE_BYTES;
-  static constexpr int KV_OFF_DO = KV_OFF_Q + KV_QS * TILE_BYTES;
-  static constexpr int KV_OFF_VEC = KV_OFF_DO + KV_QS * TILE_BYTES;  // per stage: lse2[128], D[128]
+  static constexpr int KV_OFF_DO = KV_OFF_Q + KV_QS * Q_TILE;
+  static constexpr int KV_OFF_VEC = KV_OFF_DO + KV_QS * Q_TILE;  // per stage: lse2[BMQ] at +0, D[BMQ] at +512
   static constexpr int KV_OFF_BAR = KV_OFF_VEC + KV_QS * 1024;
   static constexpr int KV_SMEM = KV_OFF_BAR + 256 + 1024;
   static_assert(DQ_SMEM <= 232448 && KV_SMEM <= 232448, "shared memory budget");
+  static_assert(DQ_KS <= 4 && DQ_VS <= 4 && KV_QS <= 3, "barrier arrays");
 };
+
+// Passes of the dK/dV kernel: both gradients (d <= 128), or dV and dK in
+// two launches (d = 256).
+constexpr int BWD_KV_BOTH = 0, BWD_KV_DV = 1, BWD_KV_DK = 2;
 
 struct BwdParams {
   const __nv_bfloat16* o;     // forward output [B*H, N, d]
@@ -108,7 +128,9 @@ struct BwdParams {
   int N;
   int d;            // head dimension of the tensors (<= HD; the kernel's tiles are zero-padded to HD)
   int BH;
-  int n_tiles;      // ceil(N / 128), for queries and keys alike
+  int n_tiles;      // ceil(N / 128): the dQ kernel's query tiles and the dK/dV kernel's key tiles
+  int n_ktiles;     // ceil(N / BNK): key tiles streamed by the dQ kernel
+  int n_qtiles;     // ceil(N / BMQ): query tiles streamed by the dK/dV kernel
   int group_heads;  // heads per launch-order group
   float scale;
   float scale_log2;
@@ -143,14 +165,15 @@ __device__ __forceinline__ void store_row32_bf16(__nv_bfloat16* dst, const uint3
                            pack_bf16x2(__uint_as_float(a[e + 6]) * f, __uint_as_float(a[e + 7]) * f));
 }
 
-// dS for 128 keys of one row: reads dP from TMEM 32 columns at a time and
-// writes dS (bf16 pairs) over the first 64 columns.  Chunk q writes packed
-// columns [16q, 16q+16), which held dP of keys 16q..16q+15: chunk q/2 <= q
-// has already read them.
-__device__ __forceinline__ void ds_to_tmem(uint32_t dp_addr, const float (&p)[128], const float* dsub, bool per_col,
+// dS for NC keys (or queries) of one row: reads dP from TMEM 32 columns at a
+// time and writes dS (bf16 pairs) over the first NC/2 columns.  Chunk q
+// writes packed columns [16q, 16q+16), which held dP of keys 16q..16q+15:
+// chunk q/2 <= q has already read them.
+template <int NC>
+__device__ __forceinline__ void ds_to_tmem(uint32_t dp_addr, const float (&p)[NC], const float* dsub, bool per_col,
                                            float dsub_row) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < NC / 32; ++q) {
     uint32_t dp[32];
     tmem_ld32(dp_addr + 32 * q, dp);
     tmem_wait_ld();
@@ -177,7 +200,7 @@ struct DqBars {
 };
 static_assert(sizeof(DqBars) <= 256, "barrier block");
 
-// TMEM columns of the dQ kernel: S [0,128), dP [128,256), dQ [256, 256+d).
+// TMEM columns of the dQ kernel: S [0,BNK), dP [128,128+BNK), dQ [256, 256+d).
 constexpr uint32_t BQ_S = 0, BQ_DP = 128, BQ_DQ = 256;
 
 template <int HD, bool CAUSAL>
@@ -186,10 +209,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                       const BwdParams p) {
   using C = BwdCfg<HD>;
+  constexpr int BNK = C::BNK;
   int bh, qt;
   bwd_item<CAUSAL, true>(p, bh, qt);
   const int q0 = qt * BM;
-  const int nkv = CAUSAL ? min(qt + 1, p.n_tiles) : p.n_tiles;
+  // Key tiles up to the one holding this query tile's last row (causal).
+  const int nkv = CAUSAL ? min((q0 + BM - 1) / BNK + 1, p.n_ktiles) : p.n_ktiles;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -254,17 +279,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             !wait_bounded(smem_u32(&bars->k_empty[ks]), ((j / C::DQ_KS) - 1) & 1, abort_flag, to, ROLE_PRODUCER))
           break;
         const uint32_t kb = smem_u32(&bars->k_full[ks]);
-        mbar_arrive_expect_tx(kb, C::TILE_BYTES);
+        mbar_arrive_expect_tx(kb, C::KV_TILE);
         for (int c = 0; c < C::KCH; ++c)
-          tma_load_3d(sK + ks * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_k, kb, c * 64, j * BN, bh);
+          tma_load_3d(sK + ks * C::KV_TILE + c * C::KV_CHUNK, &tm_k, kb, c * 64, j * BNK, bh);
         ++k_issued;
         if (j >= C::DQ_VS &&
             !wait_bounded(smem_u32(&bars->v_empty[vs]), ((j / C::DQ_VS) - 1) & 1, abort_flag, to, ROLE_PRODUCER))
           break;
         const uint32_t vb = smem_u32(&bars->v_full[vs]);
-        mbar_arrive_expect_tx(vb, C::TILE_BYTES);
+        mbar_arrive_expect_tx(vb, C::KV_TILE);
         for (int c = 0; c < C::KCH; ++c)
-          tma_load_3d(sV + vs * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_v, vb, c * 64, j * BN, bh);
+          tma_load_3d(sV + vs * C::KV_TILE + c * C::KV_CHUNK, &tm_v, vb, c * 64, j * BNK, bh);
         ++v_issued;
       }
       if (load_qdo) wait_drain(bq, 0, to);
@@ -277,14 +302,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     // S(0), dP(0); then per j >= 1: S(j), dQ(j-1), dP(j).  dS(j-1) lives in
     // dP's columns, so dP(j) is issued after dQ(j-1) has been (in order).
     if (lane == 0) {
-      constexpr uint32_t IDESC_SS = idesc_bf16_f32(BM, BN, false, false);
+      constexpr uint32_t IDESC_SS = idesc_bf16_f32(BM, BNK, false, false);
       constexpr uint32_t IDESC_DQ = idesc_bf16_f32(BM, HD, false, true);
+      // A: a 128-row tile (Q or dO); B: a BNK-row tile (K or V); both K-major.
       auto mma_kmajor = [&](uint32_t d_tmem, uint32_t a, uint32_t b) {
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-          mma_ss(d_tmem, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b + off, 16, 1024), IDESC_SS,
-                 kk > 0 ? 1u : 0u);
+          const uint32_t in_chunk = (kk & 3) * 32;
+          mma_ss(d_tmem, smem_desc_sw128(a + (kk >> 2) * C::CHUNK_BYTES + in_chunk, 16, 1024),
+                 smem_desc_sw128(b + (kk >> 2) * C::KV_CHUNK + in_chunk, 16, 1024), IDESC_SS, kk > 0 ? 1u : 0u);
         }
       };
       bool ok = wait_bounded(smem_u32(&bars->qdo_full), 0, abort_flag, to, ROLE_MMA);
@@ -309,16 +335,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                wait_bounded(smem_u32(&bars->s_free), i & 1, abort_flag, to, ROLE_MMA);
           if (!ok) break;
           tc_fence_after();
-          mma_kmajor(tmem + BQ_S, sQ, sK + ks * C::TILE_BYTES);
+          mma_kmajor(tmem + BQ_S, sQ, sK + ks * C::KV_TILE);
           mma_commit(smem_u32(&bars->s_full));
         }
         ok = wait_bounded(smem_u32(&bars->ds_ready), i & 1, abort_flag, to, ROLE_MMA);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t kbase = sK + (i % C::DQ_KS) * C::TILE_BYTES;
+        const uint32_t kbase = sK + (i % C::DQ_KS) * C::KV_TILE;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(tmem + BQ_DQ, tmem + BQ_DP + kk * 8, smem_desc_sw128(kbase + kk * 2048, C::CHUNK_BYTES, 1024),
+        for (int kk = 0; kk < BNK / 16; ++kk)
+          mma_ts(tmem + BQ_DQ, tmem + BQ_DP + kk * 8, smem_desc_sw128(kbase + kk * 2048, C::KV_CHUNK, 1024),
                  IDESC_DQ, (i > 0 || kk > 0) ? 1u : 0u);
         mma_commit(smem_u32(&bars->k_empty[i % C::DQ_KS]));
         if (j < nkv) {
@@ -326,7 +352,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           ok = wait_bounded(smem_u32(&bars->v_full[vs]), (j / C::DQ_VS) & 1, abort_flag, to, ROLE_MMA);
           if (!ok) break;
           tc_fence_after();
-          mma_kmajor(tmem + BQ_DP, sDO, sV + vs * C::TILE_BYTES);
+          mma_kmajor(tmem + BQ_DP, sDO, sV + vs * C::KV_TILE);
           mma_commit(smem_u32(&bars->dp_full));
           mma_commit(smem_u32(&bars->v_empty[vs]));
         }
@@ -369,28 +395,28 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       ok = wait_warp(smem_u32(&bars->s_full), j & 1, abort_flag, to);
       if (!ok) break;
       tc_fence_after();
-      float pr[128];
+      float pr[BNK];
       {
-        uint32_t s[128];
+        uint32_t s[BNK];
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
+        for (int cc = 0; cc < BNK / 32; ++cc)
           tmem_ld32(lane_addr + BQ_S + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
         tmem_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
+        for (int cc = 0; cc < BNK / 32; ++cc) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars->s_free));
-        const int kv0 = j * BN;
-        const bool diag = CAUSAL && (j == qt);  // key column e visible iff e <= r
-        const bool tail = !CAUSAL && (kv0 + BN > p.N);
-        const int lim = diag ? r : (p.N - 1 - kv0);  // last allowed key column
-        bwd_probs<false>(pr, s, c, nlse2, nullptr, diag || tail, lim, false);
+        const int kv0 = j * BNK;
+        const bool diag = CAUSAL && (kv0 + BNK - 1 > q0);  // the tile reaches past the first row
+        const bool tail = !CAUSAL && (kv0 + BNK > p.N);
+        const int lim = diag ? (row - kv0) : (p.N - 1 - kv0);  // last allowed key column
+        bwd_probs<false, BNK>(pr, s, c, nlse2, nullptr, diag || tail, lim, false);
       }
       ok = wait_warp(smem_u32(&bars->dp_full), j & 1, abort_flag, to);
       if (!ok) break;
       tc_fence_after();
-      ds_to_tmem(lane_addr + BQ_DP, pr, nullptr, false, dsum);
+      ds_to_tmem<BNK>(lane_addr + BQ_DP, pr, nullptr, false, dsum);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -399,17 +425,22 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     if (ok) ok = wait_warp(smem_u32(&bars->mma_final), 0, abort_flag, to);
     if (ok) {
       tc_fence_after();
-      uint32_t a[HD / 32][32];
+      __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bh) * p.N + row) * p.d;
+      // Up to 128 columns at a time (256 registers of dQ would not fit).
+      constexpr int GROUP = (HD < 128 ? HD : 128) / 32;
 #pragma unroll
-      for (int cc = 0; cc < HD / 32; ++cc) tmem_ld32(lane_addr + BQ_DQ + cc * 32, a[cc]);
-      tmem_wait_ld();
+      for (int g = 0; g < HD / 32; g += GROUP) {
+        uint32_t a[GROUP][32];
 #pragma unroll
-      for (int cc = 0; cc < HD / 32; ++cc) reg_fence32(a[cc]);
-      if (valid) {
-        __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bh) * p.N + row) * p.d;
+        for (int cc = 0; cc < GROUP; ++cc) tmem_ld32(lane_addr + BQ_DQ + (g + cc) * 32, a[cc]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < HD / 32; ++cc)
-          if (cc * 32 < p.d) store_row32_bf16(dst + cc * 32, a[cc], p.scale);
+        for (int cc = 0; cc < GROUP; ++cc) reg_fence32(a[cc]);
+        if (valid) {
+#pragma unroll
+          for (int cc = 0; cc < GROUP; ++cc)
+            if ((g + cc) * 32 < p.d) store_row32_bf16(dst + (g + cc) * 32, a[cc], p.scale);
+        }
       }
     }
   }
@@ -431,22 +462,26 @@ struct KvBars {
 };
 static_assert(sizeof(KvBars) <= 256, "barrier block");
 
-// TMEM columns of the dK/dV kernel: S^T [0,128), dP^T [128,256),
-// dV [256, 256+d), dK [256+d, 256+2d).
+// TMEM columns of the dK/dV kernel: S^T [0,BMQ), dP^T [128,128+BMQ), and
+// the accumulators from column 256: dV then dK (both gradients), or the one
+// gradient of a single pass.
 constexpr uint32_t BK_S = 0, BK_DP = 128, BK_DV = 256;
 
-template <int HD, bool CAUSAL>
+template <int HD, bool CAUSAL, int PASS>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                         const BwdParams p) {
   using C = BwdCfg<HD>;
-  constexpr uint32_t BK_DK = BK_DV + HD;
+  constexpr int BMQ = C::BMQ;
+  constexpr bool DO_DV = PASS != BWD_KV_DK, DO_DK = PASS != BWD_KV_DV;
+  static_assert(PASS == BWD_KV_BOTH ? HD <= 128 : HD == 256, "pass split only at d = 256");
+  constexpr uint32_t BK_DK = (PASS == BWD_KV_BOTH) ? BK_DV + HD : BK_DV;
   int bh, kt;
   bwd_item<CAUSAL, false>(p, bh, kt);
   const int k0 = kt * BN;
-  const int i_begin = CAUSAL ? kt : 0;  // query tiles that see this key tile
-  const int nq = p.n_tiles - i_begin;
+  const int i_begin = CAUSAL ? k0 / BMQ : 0;  // query tiles that see this key tile
+  const int nq = p.n_qtiles - i_begin;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -510,14 +545,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           break;
         const int i = i_begin + t;
         const uint32_t bq = smem_u32(&bars->q_full[s]);
-        mbar_arrive_expect_tx(bq, 2 * C::TILE_BYTES + 1024);
+        mbar_arrive_expect_tx(bq, 2 * C::Q_TILE + 2 * BMQ * 4);
         for (int c = 0; c < C::KCH; ++c) {
-          tma_load_3d(sQ + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, bq, c * 64, i * BM, bh);
-          tma_load_3d(sDO + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_do, bq, c * 64, i * BM, bh);
+          tma_load_3d(sQ + s * C::Q_TILE + c * C::Q_CHUNK, &tm_q, bq, c * 64, i * BMQ, bh);
+          tma_load_3d(sDO + s * C::Q_TILE + c * C::Q_CHUNK, &tm_do, bq, c * 64, i * BMQ, bh);
         }
         const uint32_t sv = base + C::KV_OFF_VEC + s * 1024;
-        bulk_load_1d(sv, p.lse2 + vec_head + i * BM, 512, bq);
-        bulk_load_1d(sv + 512, p.dvec + vec_head + i * BM, 512, bq);
+        bulk_load_1d(sv, p.lse2 + vec_head + i * BMQ, BMQ * 4, bq);
+        bulk_load_1d(sv + 512, p.dvec + vec_head + i * BMQ, BMQ * 4, bq);
         ++issued;
       }
       if (load_kv) wait_drain(bkv, 0, to);
@@ -525,24 +560,27 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         wait_drain(smem_u32(&bars->q_full[x % C::KV_QS]), (x / C::KV_QS) & 1, to);
     }
   } else if (warp == BWD_MMA_WARP) {
-    // S^T(0), dP^T(0); then per query tile t: dV(t), S^T(t+1), dK(t),
-    // dP^T(t+1).  P^T(t) lives in S^T's columns and dS^T(t) in dP^T's, so
-    // each overwrite is issued after the MMA that reads them (in order).
+    // Both gradients: S^T(0), dP^T(0); then per query tile t: dV(t),
+    // S^T(t+1), dK(t), dP^T(t+1).  dV pass: S^T(0); then dV(t), S^T(t+1).
+    // dK pass: S^T(0), dP^T(0); then dK(t), S^T(t+1), dP^T(t+1).  P^T(t)
+    // lives in S^T's columns and dS^T(t) in dP^T's, so each overwrite is
+    // issued after the MMA that reads them (in order).
     if (lane == 0) {
-      constexpr uint32_t IDESC_SS = idesc_bf16_f32(BN, BM, false, false);
+      constexpr uint32_t IDESC_SS = idesc_bf16_f32(BN, BMQ, false, false);
       constexpr uint32_t IDESC_ACC = idesc_bf16_f32(BN, HD, false, true);
+      // A: the 128-row K or V tile; B: a BMQ-row Q or dO tile; both K-major.
       auto mma_kmajor = [&](uint32_t d_tmem, uint32_t a, uint32_t b) {
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-          mma_ss(d_tmem, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b + off, 16, 1024), IDESC_SS,
-                 kk > 0 ? 1u : 0u);
+          const uint32_t in_chunk = (kk & 3) * 32;
+          mma_ss(d_tmem, smem_desc_sw128(a + (kk >> 2) * C::CHUNK_BYTES + in_chunk, 16, 1024),
+                 smem_desc_sw128(b + (kk >> 2) * C::Q_CHUNK + in_chunk, 16, 1024), IDESC_SS, kk > 0 ? 1u : 0u);
         }
       };
       auto mma_acc = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b, bool acc) {
 #pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b + kk * 2048, C::CHUNK_BYTES, 1024), IDESC_ACC,
+        for (int kk = 0; kk < BMQ / 16; ++kk)
+          mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b + kk * 2048, C::Q_CHUNK, 1024), IDESC_ACC,
                  (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = wait_bounded(smem_u32(&bars->kv_full), 0, abort_flag, to, ROLE_MMA) &&
@@ -551,31 +589,46 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         tc_fence_after();
         mma_kmajor(tmem + BK_S, sK, sQ);
         mma_commit(smem_u32(&bars->s_full));
-        mma_kmajor(tmem + BK_DP, sV, sDO);
-        mma_commit(smem_u32(&bars->dp_full));
+        if constexpr (DO_DK) {
+          mma_kmajor(tmem + BK_DP, sV, sDO);
+          mma_commit(smem_u32(&bars->dp_full));
+        }
       }
       for (int t = 0; ok && t < nq; ++t) {
         const int s = t % C::KV_QS;
-        ok = wait_bounded(smem_u32(&bars->p_ready), t & 1, abort_flag, to, ROLE_MMA);
-        if (!ok) break;
-        tc_fence_after();
-        mma_acc(tmem + BK_DV, tmem + BK_S, sDO + s * C::TILE_BYTES, t > 0);
         const bool more = t + 1 < nq;
         const int s1 = (t + 1) % C::KV_QS;
+        if constexpr (DO_DV) {
+          ok = wait_bounded(smem_u32(&bars->p_ready), t & 1, abort_flag, to, ROLE_MMA);
+          if (!ok) break;
+          tc_fence_after();
+          mma_acc(tmem + BK_DV, tmem + BK_S, sDO + s * C::Q_TILE, t > 0);
+          // dV pass: the stage's last reader was just issued (the producer
+          // may then refill it, which the next S^T waits for).
+          if constexpr (PASS == BWD_KV_DV) mma_commit(smem_u32(&bars->q_empty[s]));
+        } else {
+          ok = wait_bounded(smem_u32(&bars->ds_ready), t & 1, abort_flag, to, ROLE_MMA);
+          if (!ok) break;
+          tc_fence_after();
+          mma_acc(tmem + BK_DK, tmem + BK_DP, sQ + s * C::Q_TILE, t > 0);
+          mma_commit(smem_u32(&bars->q_empty[s]));
+        }
         if (more) {
           ok = wait_bounded(smem_u32(&bars->q_full[s1]), ((t + 1) / C::KV_QS) & 1, abort_flag, to, ROLE_MMA);
           if (!ok) break;
           tc_fence_after();
-          mma_kmajor(tmem + BK_S, sK, sQ + s1 * C::TILE_BYTES);
+          mma_kmajor(tmem + BK_S, sK, sQ + s1 * C::Q_TILE);
           mma_commit(smem_u32(&bars->s_full));
         }
-        ok = wait_bounded(smem_u32(&bars->ds_ready), t & 1, abort_flag, to, ROLE_MMA);
-        if (!ok) break;
-        tc_fence_after();
-        mma_acc(tmem + BK_DK, tmem + BK_DP, sQ + s * C::TILE_BYTES, t > 0);
-        mma_commit(smem_u32(&bars->q_empty[s]));
-        if (more) {
-          mma_kmajor(tmem + BK_DP, sV, sDO + s1 * C::TILE_BYTES);
+        if constexpr (PASS == BWD_KV_BOTH) {
+          ok = wait_bounded(smem_u32(&bars->ds_ready), t & 1, abort_flag, to, ROLE_MMA);
+          if (!ok) break;
+          tc_fence_after();
+          mma_acc(tmem + BK_DK, tmem + BK_DP, sQ + s * C::Q_TILE, t > 0);
+          mma_commit(smem_u32(&bars->q_empty[s]));
+        }
+        if (DO_DK && more) {
+          mma_kmajor(tmem + BK_DP, sV, sDO + s1 * C::Q_TILE);
           mma_commit(smem_u32(&bars->dp_full));
         }
       }
@@ -596,61 +649,71 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
            wait_warp(smem_u32(&bars->q_full[s]), (t / C::KV_QS) & 1, abort_flag, to);
       if (!ok) break;
       tc_fence_after();
-      const float* l2 = vec + s * 256;  // -LSE*log2(e) of the tile's 128 queries (-inf past N)
-      const float* dd = l2 + 128;       // D of the tile's 128 queries
-      float pr[128];
+      const float* l2 = vec + s * 256;  // -LSE*log2(e) of the tile's BMQ queries (-inf past N)
+      const float* dd = l2 + 128;       // D of the tile's BMQ queries
+      float pr[BMQ];
       {
-        uint32_t sv[128];
+        uint32_t sv[BMQ];
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
+        for (int cc = 0; cc < BMQ / 32; ++cc)
           tmem_ld32(lane_addr + BK_S + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
         tmem_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
-        const bool diag = CAUSAL && (i == kt);  // query 128i + e sees this key only if e >= r
-        bwd_probs<true>(pr, sv, c, 0.f, l2, diag, r, true);
+        for (int cc = 0; cc < BMQ / 32; ++cc) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sv[cc * 32]));
+        // Query i*BMQ + e sees this key only if i*BMQ + e >= key.
+        const int q_first = i * BMQ;
+        const bool diag = CAUSAL && (q_first < k0 + BN - 1);
+        bwd_probs<true, BMQ>(pr, sv, c, 0.f, l2, diag, key - q_first, true);
       }
-      // P^T (bf16) over the first 64 score columns, for dV += P^T dO.
+      if constexpr (DO_DV) {
+        // P^T (bf16) over the first BMQ/2 score columns, for dV += P^T dO.
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
+        for (int h = 0; h < BMQ / 64; ++h) {
+          uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pr[64 * h + 2 * e], pr[64 * h + 2 * e + 1]);
-        tmem_st32(lane_addr + BK_S + 32 * h, pk);
+          for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pr[64 * h + 2 * e], pr[64 * h + 2 * e + 1]);
+          tmem_st32(lane_addr + BK_S + 32 * h, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready));
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready));
-      ok = wait_warp(smem_u32(&bars->dp_full), t & 1, abort_flag, to);
-      if (!ok) break;
-      tc_fence_after();
-      ds_to_tmem(lane_addr + BK_DP, pr, dd, true, 0.f);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->ds_ready));
+      if constexpr (DO_DK) {
+        ok = wait_warp(smem_u32(&bars->dp_full), t & 1, abort_flag, to);
+        if (!ok) break;
+        tc_fence_after();
+        ds_to_tmem<BMQ>(lane_addr + BK_DP, pr, dd, true, 0.f);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->ds_ready));
+      }
     }
     if (ok) ok = wait_warp(smem_u32(&bars->mma_final), 0, abort_flag, to);
     if (ok) {
       tc_fence_after();
       const bool valid = key < p.N;
       const size_t off = (static_cast<size_t>(bh) * p.N + key) * p.d;
+      if constexpr (DO_DV) {
 #pragma unroll
-      for (int cc = 0; cc < HD / 32; ++cc) {
-        uint32_t a[32];
-        tmem_ld32(lane_addr + BK_DV + cc * 32, a);
-        tmem_wait_ld();
-        reg_fence32(a);
-        if (valid && cc * 32 < p.d) store_row32_bf16(p.dv + off + cc * 32, a, 1.f);
+        for (int cc = 0; cc < HD / 32; ++cc) {
+          uint32_t a[32];
+          tmem_ld32(lane_addr + BK_DV + cc * 32, a);
+          tmem_wait_ld();
+          reg_fence32(a);
+          if (valid && cc * 32 < p.d) store_row32_bf16(p.dv + off + cc * 32, a, 1.f);
+        }
       }
+      if constexpr (DO_DK) {
 #pragma unroll
-      for (int cc = 0; cc < HD / 32; ++cc) {
-        uint32_t a[32];
-        tmem_ld32(lane_addr + BK_DK + cc * 32, a);
-        tmem_wait_ld();
-        reg_fence32(a);
-        if (valid && cc * 32 < p.d) store_row32_bf16(p.dk + off + cc * 32, a, p.scale);
+        for (int cc = 0; cc < HD / 32; ++cc) {
+          uint32_t a[32];
+          tmem_ld32(lane_addr + BK_DK + cc * 32, a);
+          tmem_wait_ld();
+          reg_fence32(a);
+          if (valid && cc * 32 < p.d) store_row32_bf16(p.dk + off + cc * 32, a, p.scale);
+        }
       }
     }
   }

@@ -1028,9 +1028,26 @@ static size_t bwd_workspace_bytes_for(int B, int H, int N) {
   return 2 * round256(rows * 4);
 }
 
+template <typename Kern>
+static int bwd_set_smem(Kern kern, int bytes) {
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) {
+    set_detail("cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    return FA2_ERR_CUDA;
+  }
+  return FA2_OK;
+}
+
+// Maps: the dQ kernel reads 128-row Q and dO tiles and BNK-row K and V
+// tiles; the dK/dV kernel 128-row K and V tiles and BMQ-row Q and dO tiles
+// (the same maps when both are 128, i.e. d <= 128).
+struct BwdMaps {
+  CUtensorMap q128, do128, k_dq, v_dq;  // dQ kernel
+  CUtensorMap k128, v128, q_kv, do_kv;  // dK/dV kernel(s)
+};
+
 template <int HD, bool CAUSAL>
-static int bwd_launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                        const BwdParams& prm, cudaStream_t stream) {
+static int bwd_launch_t(const BwdMaps& m, const BwdParams& prm, cudaStream_t stream) {
   using C = BwdCfg<HD>;
   static std::atomic<unsigned> attr_done_mask{0};  // per device bit (devices 0..31)
   int dev = 0;
@@ -1038,29 +1055,38 @@ static int bwd_launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
     set_detail("cudaGetDevice failed");
     return FA2_ERR_CUDA;
   }
+  constexpr int PASS0 = (HD == 256) ? BWD_KV_DV : BWD_KV_BOTH;
   auto kq = fa2_bwd_dq_kernel<HD, CAUSAL>;
-  auto kkv = fa2_bwd_dkdv_kernel<HD, CAUSAL>;
+  auto kkv = fa2_bwd_dkdv_kernel<HD, CAUSAL, PASS0>;
   if (dev >= 32 || !(attr_done_mask.load(std::memory_order_acquire) & (1u << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::DQ_SMEM);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, C::KV_SMEM);
-    if (e != cudaSuccess) {
-      set_detail("cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-      return FA2_ERR_CUDA;
-    }
+    int st = bwd_set_smem(kq, C::DQ_SMEM);
+    if (st == FA2_OK) st = bwd_set_smem(kkv, C::KV_SMEM);
+    if constexpr (HD == 256)
+      if (st == FA2_OK) st = bwd_set_smem(fa2_bwd_dkdv_kernel<HD, CAUSAL, BWD_KV_DK>, C::KV_SMEM);
+    if (st != FA2_OK) return st;
     if (dev < 32) attr_done_mask.fetch_or(1u << dev, std::memory_order_acq_rel);
   }
   const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_tiles);
-  kq<<<grid, BWD_THREADS, C::DQ_SMEM, stream>>>(tq, tk, tv, tdo, prm);
+  kq<<<grid, BWD_THREADS, C::DQ_SMEM, stream>>>(m.q128, m.k_dq, m.v_dq, m.do128, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_detail("dQ kernel launch: %s", cudaGetErrorString(e));
     return FA2_ERR_CUDA;
   }
-  kkv<<<grid, BWD_THREADS, C::KV_SMEM, stream>>>(tq, tk, tv, tdo, prm);
+  kkv<<<grid, BWD_THREADS, C::KV_SMEM, stream>>>(m.q_kv, m.k128, m.v128, m.do_kv, prm);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_detail("dK/dV kernel launch: %s", cudaGetErrorString(e));
     return FA2_ERR_CUDA;
+  }
+  if constexpr (HD == 256) {
+    fa2_bwd_dkdv_kernel<HD, CAUSAL, BWD_KV_DK><<<grid, BWD_THREADS, C::KV_SMEM, stream>>>(m.q_kv, m.k128, m.v128,
+                                                                                         m.do_kv, prm);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      set_detail("dK kernel launch: %s", cudaGetErrorString(e));
+      return FA2_ERR_CUDA;
+    }
   }
   return FA2_OK;
 }
@@ -1083,8 +1109,8 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
     set_detail("scale must be finite and positive");
     return FA2_ERR_INVALID_ARG;
   }
-  if (!d_supported(d) || padded_hd(d) == 256) {
-    set_detail("head dimension %d not supported by the backward (32, 64, 96 or 128)", d);
+  if (!d_supported(d)) {
+    set_detail("head dimension %d not supported (32, 64, 96, 128 or 256)", d);
     return FA2_ERR_UNSUPPORTED;
   }
   const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
@@ -1118,17 +1144,26 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
         return FA2_ERR_INVALID_ARG;
       }
   }
-  CUtensorMap tq, tk, tv, tdo;
+  // d = 256: 64-key tiles in the dQ kernel, 64-query tiles in the dK/dV kernels.
+  const int tile_small = padded_hd(d) == 256 ? 64 : 128;
+  BwdMaps maps;
   int st;
-  if ((st = make_tmap(&tq, q, d, N, static_cast<int>(BH))) != FA2_OK) return st;
-  if ((st = make_tmap(&tk, k, d, N, static_cast<int>(BH))) != FA2_OK) return st;
-  if ((st = make_tmap(&tv, v, d, N, static_cast<int>(BH))) != FA2_OK) return st;
-  if ((st = make_tmap(&tdo, dout, d, N, static_cast<int>(BH))) != FA2_OK) return st;
+  const int bhi = static_cast<int>(BH);
+  if ((st = make_tmap(&maps.q128, q, d, N, bhi)) != FA2_OK) return st;
+  if ((st = make_tmap(&maps.do128, dout, d, N, bhi)) != FA2_OK) return st;
+  if ((st = make_tmap(&maps.k128, k, d, N, bhi)) != FA2_OK) return st;
+  if ((st = make_tmap(&maps.v128, v, d, N, bhi)) != FA2_OK) return st;
+  if ((st = make_tmap(&maps.k_dq, k, d, N, bhi, tile_small)) != FA2_OK) return st;
+  if ((st = make_tmap(&maps.v_dq, v, d, N, bhi, tile_small)) != FA2_OK) return st;
+  if ((st = make_tmap(&maps.q_kv, q, d, N, bhi, tile_small)) != FA2_OK) return st;
+  if ((st = make_tmap(&maps.do_kv, dout, d, N, bhi, tile_small)) != FA2_OK) return st;
   BwdParams prm;
   prm.o = static_cast<const __nv_bfloat16*>(o);
   prm.dout = static_cast<const __nv_bfloat16*>(dout);
   prm.lse = lse;
   prm.n_tiles = (N + BM - 1) / BM;
+  prm.n_ktiles = (N + tile_small - 1) / tile_small;
+  prm.n_qtiles = (N + tile_small - 1) / tile_small;
   prm.lse2 = static_cast<float*>(workspace);
   prm.dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) + need / 2);
   prm.dq = static_cast<__nv_bfloat16*>(dq);
@@ -1143,10 +1178,10 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   prm.timeout_ns = timeout_ns;
   prm.inject_timeout = inject;
   if (padded_hd(d) == 64)
-    return causal ? bwd_launch_t<64, true>(tq, tk, tv, tdo, prm, stream)
-                  : bwd_launch_t<64, false>(tq, tk, tv, tdo, prm, stream);
-  return causal ? bwd_launch_t<128, true>(tq, tk, tv, tdo, prm, stream)
-                : bwd_launch_t<128, false>(tq, tk, tv, tdo, prm, stream);
+    return causal ? bwd_launch_t<64, true>(maps, prm, stream) : bwd_launch_t<64, false>(maps, prm, stream);
+  if (padded_hd(d) == 256)
+    return causal ? bwd_launch_t<256, true>(maps, prm, stream) : bwd_launch_t<256, false>(maps, prm, stream);
+  return causal ? bwd_launch_t<128, true>(maps, prm, stream) : bwd_launch_t<128, false>(maps, prm, stream);
 }
 
 // ------------------------------------------------------------------ split-K/V with library-owned scratch
@@ -1394,7 +1429,7 @@ int fa2_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o,
 }
 
 size_t fa2_bwd_workspace_bytes(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || !fa2::d_supported(d) || fa2::padded_hd(d) == 256) return 0;
+  if (B < 1 || H < 1 || N < 1 || !fa2::d_supported(d)) return 0;
   return fa2::bwd_workspace_bytes_for(B, H, N);
 }
 

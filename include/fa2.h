@@ -203,14 +203,17 @@ size_t fa2_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int 
  *   lse     : device pointer, fp32 [B,H,N], natural log, 4-byte aligned.
  *   dq, dk, dv : device pointers, bf16 [B,H,N,d]; written.  They must not
  *             overlap each other, the inputs or the workspace.
- *   B, H, N, d, causal, scale : as for fa2_fwd, but d 32, 64, 96 or 128
- *             (256 -> FA2_ERR_UNSUPPORTED); scale > 0.
+ *   B, H, N, d, causal, scale : as for fa2_fwd (d 32, 64, 96, 128 or 256;
+ *             scale > 0).
  *   workspace, workspace_bytes : caller-owned device buffer, 256-byte
  *             aligned, of at least fa2_bwd_workspace_bytes(B,H,N,d) bytes;
  *             it carries per-row -LSE*log2(e) and rowsum(dO o O) from the
  *             first kernel to the second.  Concurrent calls need separate
  *             workspaces.
- *   stream  : cudaStream_t as void*; two kernels are queued on it.
+ *   stream  : cudaStream_t as void*; two kernels are queued on it (three
+ *             at d = 256: the dQ kernel streams 64-key tiles, and dV and dK
+ *             are computed by two passes over 64-query tiles, since their
+ *             accumulators and the two score tiles exceed tensor memory).
  * Argument errors are reported before anything is launched; kernel-side
  * timeouts through fa2_sync_status.
  */
@@ -225,7 +228,7 @@ size_t fa2_bwd_workspace_bytes(int B, int H, int N, int d);
  * Test hook for the failure path of fa2_bwd (same arguments, plus `kernel`
  * and `timeout_ns`, 1 .. 2e9).  kernel = 0: the dQ kernel runs with its Q/dO
  * tile load withheld; kernel = 1: the dK/dV kernel runs with its K/V tile load
- * withheld.  That kernel's waits run out after `timeout_ns`; it records the
+ * withheld (both passes at d = 256).  That kernel's waits run out after `timeout_ns`; it records the
  * time-out, drains its own copies and MMAs, releases tensor memory and
  * returns; the other kernel runs normally.  fa2_sync_status returns
  * FA2_ERR_TIMEOUT.  Gradients are unspecified.  kernel outside {0, 1} ->

@@ -245,7 +245,7 @@ def test_bwd_workspace_size(lib):
     assert lib.fa2_bwd_workspace_bytes(1, 1, 1, 64) == 2 * 512
     assert lib.fa2_bwd_workspace_bytes(1, 1, 0, 64) == 0
     assert lib.fa2_bwd_workspace_bytes(1, 1, 8, 80) == 0
-    assert lib.fa2_bwd_workspace_bytes(1, 1, 8, 256) == 0  # the backward serves d <= 128
+    assert lib.fa2_bwd_workspace_bytes(1, 1, 8, 256) == 2 * 512  # d = 256 too (64-key / 64-query tiles)
     assert lib.fa2_bwd_workspace_bytes(1, 1, 8, 96) == 2 * 512  # d = 96 runs on zero-padded 128-column tiles
 
 
@@ -255,7 +255,7 @@ def test_bwd_workspace_size(lib):
     (dict(ws=0), binding.FA2_ERR_INVALID_ARG),
     (dict(N=0), binding.FA2_ERR_INVALID_ARG),
     (dict(d=80), binding.FA2_ERR_UNSUPPORTED),
-    (dict(d=256), binding.FA2_ERR_UNSUPPORTED),
+    (dict(d=512), binding.FA2_ERR_UNSUPPORTED),
     (dict(scale=0.0), binding.FA2_ERR_INVALID_ARG),
     (dict(scale=float("inf")), binding.FA2_ERR_INVALID_ARG),
     (dict(ws=FAKE + (9 << 32) + 64), binding.FA2_ERR_INVALID_ARG),   # workspace not 256-aligned

@@ -72,7 +72,7 @@ def test_splitkv_withheld_load_times_out_and_context_survives(B, H, Nq, Nk, d, c
 
 
 @pytest.mark.parametrize("kernel", [0, 1], ids=["dq_kernel", "dkdv_kernel"])
-@pytest.mark.parametrize("d,causal", [(64, True), (128, False)])
+@pytest.mark.parametrize("d,causal", [(64, True), (128, False), (256, True)])
 def test_backward_withheld_load_times_out_and_context_survives(kernel, d, causal):
     B, H, N = 1, 2, 300
     q, k, v = make_qkv(B, H, N, d, seed=5)
