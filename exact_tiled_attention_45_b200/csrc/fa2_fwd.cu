@@ -898,7 +898,7 @@ static size_t skv_workspace_bytes(int B, int H, int Nq, int d, int splits) {
 template <int HD, bool CAUSAL, bool QUAD>
 static int skv_launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const SkvParams& prm,
                         int n_q_tiles, int splits, __nv_bfloat16* o, float* lse, cudaStream_t stream) {
-  using C = SkvCfg<HD>;
+  using C = SkvCfg<HD, skv_slim<HD, QUAD>()>;
   auto kern = fa2_splitkv_kernel<HD, CAUSAL, QUAD>;
   static std::atomic<unsigned> attr_done_mask{0};  // per device bit (devices 0..31)
   int dev = 0;

@@ -44,7 +44,19 @@ constexpr int SKV_THREADS = 192;
 constexpr int SKV_PRODUCER_WARP = 4;
 constexpr int SKV_MMA_WARP = 5;
 
-template <int HD>
+// Slim configuration (d = 64, quarter mode): 2-stage K and V rings (80 KB
+// of shared memory with the query tile), one score and one P buffer (256
+// TMEM columns), so that two CTAs share an SM and one's set-up, hand-offs
+// and tail overlap the other's stream of keys.
+#ifndef FA2_SKV_SLIM_D64
+#define FA2_SKV_SLIM_D64 1
+#endif
+template <int HD, bool QUAD>
+__host__ __device__ constexpr bool skv_slim() {
+  return FA2_SKV_SLIM_D64 && HD == 64 && QUAD;
+}
+
+template <int HD, bool SLIM = false>
 struct SkvCfg {
   static constexpr int SBN = (HD == 256) ? 64 : 128;  // keys per tile
   static constexpr int KCH = HD / 64;                 // 64-column (128-byte) chunks
@@ -55,7 +67,7 @@ struct SkvCfg {
   // Deep K/V rings: the stream over keys is the bound for few queries, so
   // keep many tiles in flight (224 KB of rings for d = 128, 128 KB for d = 64,
   // 128 KB for d = 256).
-  static constexpr int KS = (HD == 64) ? 4 : (HD == 128 ? 3 : 2);
+  static constexpr int KS = SLIM ? 2 : (HD == 64) ? 4 : (HD == 128 ? 3 : 2);
   static constexpr int VS = KS;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
@@ -63,10 +75,17 @@ struct SkvCfg {
   static constexpr int OFF_BAR = OFF_V + VS * KV_BYTES;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  // TMEM columns: S0, S1 (SBN each), P0, P1 (SBN/2 packed bf16 pairs each), O (HD).
-  static constexpr uint32_t TM_S0 = 0, TM_S1 = SBN, TM_P = 2 * SBN, TM_O = (HD == 256) ? 256 : 384;
+  static_assert(!SLIM || 2 * (SMEM_BYTES + 1024) <= 233472, "two slim CTAs per SM");
+  static constexpr int MIN_BLOCKS = SLIM ? 2 : 1;  // CTAs per SM
+  static constexpr int NSB = SLIM ? 1 : 2;          // score buffers
+  static constexpr int NPB = SLIM ? 1 : 2;          // P buffers
+  // TMEM columns: S0, S1 (SBN each), P0, P1 (SBN/2 packed bf16 pairs each), O (HD);
+  // slim: S, P, O in 256 columns.
+  static constexpr uint32_t TMEM_ALLOC = SLIM ? 256 : 512;
+  static constexpr uint32_t TM_S0 = 0, TM_S1 = SLIM ? 0 : SBN, TM_P = NSB * SBN;
+  static constexpr uint32_t TM_O = SLIM ? TM_P + SBN / 2 : (HD == 256) ? 256 : 384;
   __host__ __device__ static constexpr uint32_t tm_p(int b) { return TM_P + static_cast<uint32_t>(b) * (SBN / 2); }
-  static_assert(TM_P + SBN <= TM_O && TM_O + HD <= 512, "TMEM budget");
+  static_assert(TM_P + NPB * SBN / 2 <= TM_O && TM_O + HD <= TMEM_ALLOC, "TMEM budget");
 };
 
 struct SkvParams {
@@ -100,10 +119,10 @@ struct SkvBarriers {
 static_assert(sizeof(SkvBarriers) <= 256, "barrier block");
 
 template <int HD, bool CAUSAL, bool QUAD>
-__global__ void __launch_bounds__(SKV_THREADS, 1)
+__global__ void __launch_bounds__(SKV_THREADS, (SkvCfg<HD, skv_slim<HD, QUAD>()>::MIN_BLOCKS))
     fa2_splitkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const SkvParams p) {
-  using C = SkvCfg<HD>;
+  using C = SkvCfg<HD, skv_slim<HD, QUAD>()>;
   static_assert(!QUAD || C::SBN == 128, "quarter mode needs 128-key tiles");
   const int q_first = static_cast<int>(blockIdx.x) * BM;
   const int bh = static_cast<int>(blockIdx.y);
@@ -169,7 +188,7 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
     fence_mbar_init();
   }
   if (warp == SKV_MMA_WARP) {
-    tmem_alloc(smem_u32(&bars->tmem_base), TMEM_COLS);
+    tmem_alloc(smem_u32(&bars->tmem_base), C::TMEM_ALLOC);
     tmem_relinquish();
   }
   if (warp == SKV_PRODUCER_WARP && lane == 0) {
@@ -238,9 +257,10 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
       for (int j = 0; ok && j <= nkv; ++j) {
         if (j < nkv) {
           const int ks = j % C::KS;
-          const int sb = j & 1;
+          const int sb = j % C::NSB;
           if (!wait_bounded(smem_u32(&bars->k_full[ks]), (j / C::KS) & 1, abort_flag, to, ROLE_MMA)) break;
-          if (j >= 2 && !wait_bounded(smem_u32(&bars->s_free[sb]), ((j - 2) >> 1) & 1, abort_flag, to, ROLE_MMA))
+          if (j >= C::NSB &&
+              !wait_bounded(smem_u32(&bars->s_free[sb]), ((j - C::NSB) / C::NSB) & 1, abort_flag, to, ROLE_MMA))
             break;
           tc_fence_after();
           const uint32_t d_s = tmem + (sb ? C::TM_S1 : C::TM_S0);
@@ -257,8 +277,8 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
         if (j >= 1) {
           const int i = j - 1;
           const int vs = i % C::VS;
-          const int pb = i & 1;
-          if (!wait_bounded(smem_u32(&bars->p_full[pb]), (i >> 1) & 1, abort_flag, to, ROLE_MMA)) break;
+          const int pb = i % C::NPB;
+          if (!wait_bounded(smem_u32(&bars->p_full[pb]), (i / C::NPB) & 1, abort_flag, to, ROLE_MMA)) break;
           if (!wait_bounded(smem_u32(&bars->v_full[vs]), (i / C::VS) & 1, abort_flag, to, ROLE_MMA)) break;
           tc_fence_after();
           const uint32_t vbase = sV + vs * C::KV_BYTES;
@@ -288,15 +308,17 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
       for (int e = 0; e < 32; ++e) z[e] = 0u;
       tmem_st32(lane_addr + C::tm_p(0), z);
       tmem_st32(lane_addr + C::tm_p(0) + 32, z);
-      tmem_st32(lane_addr + C::tm_p(1), z);
-      tmem_st32(lane_addr + C::tm_p(1) + 32, z);
+      if constexpr (C::NPB == 2) {
+        tmem_st32(lane_addr + C::tm_p(1), z);
+        tmem_st32(lane_addr + C::tm_p(1) + 32, z);
+      }
       tmem_wait_st();
     }
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int i = 0; i < nkv; ++i) {
-      const int sb = i & 1;
-      ok = wait_warp(smem_u32(&bars->s_full[sb]), (i >> 1) & 1, abort_flag, to);
+      const int sb = i % C::NSB;
+      ok = wait_warp(smem_u32(&bars->s_full[sb]), (i / C::NSB) & 1, abort_flag, to);
       if (!ok) break;
       tc_fence_after();
       const int kv0 = (kt_begin + i) * C::SBN + col0;
@@ -345,18 +367,21 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
       f2_unpack(f2_add(acc[0], acc[1]), r0, r1);
       f2_unpack(f2_add(acc[2], acc[3]), r2, r3);
       const float rowsum = (r0 + r1) + (r2 + r3);
-      const int pb = i & 1;
-      // P buffer pb was last read by PV(i-2); O is accumulated by PV(i-1),
-      // which must be complete only when O is rescaled here.
-      if (i >= 2) {
-        ok = wait_warp(smem_u32(&bars->pv_done[pb]), ((i - 2) >> 1) & 1, abort_flag, to);
+      const int pb = i % C::NPB;
+      // P buffer pb was last read by PV(i - NPB); O is accumulated by
+      // PV(i-1), which must be complete only when O is rescaled here (with one
+      // P buffer the first wait already covers it).
+      if (i >= C::NPB) {
+        ok = wait_warp(smem_u32(&bars->pv_done[pb]), ((i - C::NPB) / C::NPB) & 1, abort_flag, to);
         if (!ok) break;
         tc_fence_after();
       }
       if (i > 0 && __any_sync(0xffffffffu, rescale)) {
-        ok = wait_warp(smem_u32(&bars->pv_done[pb ^ 1]), ((i - 1) >> 1) & 1, abort_flag, to);
-        if (!ok) break;
-        tc_fence_after();
+        if constexpr (C::NPB == 2) {
+          ok = wait_warp(smem_u32(&bars->pv_done[pb ^ 1]), ((i - 1) >> 1) & 1, abort_flag, to);
+          if (!ok) break;
+          tc_fence_after();
+        }
         {
           const uint64_t aa = f2_pack(alpha, alpha);
 #pragma unroll
@@ -384,16 +409,18 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
       l = l * alpha + rowsum;
       m = m_new;
     }
-    if (ok) ok = wait_warp(smem_u32(&bars->pv_done[(nkv - 1) & 1]), ((nkv - 1) >> 1) & 1, abort_flag, to);
+    if (ok) ok = wait_warp(smem_u32(&bars->pv_done[(nkv - 1) % C::NPB]), ((nkv - 1) / C::NPB) & 1, abort_flag, to);
     // Merge of the four quarters.  Every softmax warp reaches both named
     // barriers whatever happened above (after a time-out the values are
-    // unspecified, as documented, but no warp is left waiting).  The K ring
-    // is idle here: its last reader, an S MMA, completed before the final PV.
+    // unspecified, as documented, but no warp is left waiting).  The K and V
+    // rings are idle here: their last readers, the final S and P V MMAs,
+    // completed before the final pv_done.
     constexpr int OST = HD + 4;  // padded row stride (floats) of the exchange buffer
-    float* xo = reinterpret_cast<float*>(smem + C::OFF_K);  // [4 warps][32 rows][OST]
-    float* xm = reinterpret_cast<float*>(smem + C::OFF_V);  // [4][32] running max (log2)
-    float* xl = xm + 128;                                   // [4][32] running sum
-    static_assert(4 * 32 * OST * 4 <= C::KS * C::KV_BYTES, "exchange buffer");
+    constexpr int XO_BYTES = 4 * 32 * OST * 4;
+    float* xo = reinterpret_cast<float*>(smem + C::OFF_K);             // [4 warps][32 rows][OST]
+    float* xm = reinterpret_cast<float*>(smem + C::OFF_K + XO_BYTES);  // [4][32] running max (log2)
+    float* xl = xm + 128;                                              // [4][32] running sum
+    static_assert(C::OFF_K + XO_BYTES + 2 * 128 * 4 <= C::OFF_BAR, "exchange buffer");
     xm[warp * 32 + lane] = m;
     xl[warp * 32 + lane] = l;
     named_barrier(1, 128);
@@ -480,8 +507,8 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int i = 0; i < nkv; ++i) {
-      const int sb = i & 1;
-      ok = wait_warp(smem_u32(&bars->s_full[sb]), (i >> 1) & 1, abort_flag, to);
+      const int sb = i % C::NSB;
+      ok = wait_warp(smem_u32(&bars->s_full[sb]), (i / C::NSB) & 1, abort_flag, to);
       if (!ok) break;
       tc_fence_after();
       constexpr int SBN = C::SBN;
@@ -548,18 +575,21 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars->s_free[sb]));
       }
-      const int pb = i & 1;
-      // P buffer pb was last read by PV(i-2); O is accumulated by PV(i-1),
-      // which must be complete only when O is rescaled here.
-      if (i >= 2) {
-        ok = wait_warp(smem_u32(&bars->pv_done[pb]), ((i - 2) >> 1) & 1, abort_flag, to);
+      const int pb = i % C::NPB;
+      // P buffer pb was last read by PV(i - NPB); O is accumulated by
+      // PV(i-1), which must be complete only when O is rescaled here (with one
+      // P buffer the first wait already covers it).
+      if (i >= C::NPB) {
+        ok = wait_warp(smem_u32(&bars->pv_done[pb]), ((i - C::NPB) / C::NPB) & 1, abort_flag, to);
         if (!ok) break;
         tc_fence_after();
       }
       if (i > 0 && live && __any_sync(0xffffffffu, rescale)) {
-        ok = wait_warp(smem_u32(&bars->pv_done[pb ^ 1]), ((i - 1) >> 1) & 1, abort_flag, to);
-        if (!ok) break;
-        tc_fence_after();
+        if constexpr (C::NPB == 2) {
+          ok = wait_warp(smem_u32(&bars->pv_done[pb ^ 1]), ((i - 1) >> 1) & 1, abort_flag, to);
+          if (!ok) break;
+          tc_fence_after();
+        }
         {
           const uint64_t aa = f2_pack(alpha, alpha);
 #pragma unroll
@@ -590,7 +620,7 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
       l = l * alpha + rowsum;
       m = m_new;
     }
-    if (ok) ok = wait_warp(smem_u32(&bars->pv_done[(nkv - 1) & 1]), ((nkv - 1) >> 1) & 1, abort_flag, to);
+    if (ok) ok = wait_warp(smem_u32(&bars->pv_done[(nkv - 1) % C::NPB]), ((nkv - 1) / C::NPB) & 1, abort_flag, to);
     if (ok && live) {
       tc_fence_after();
       const bool store = row < p.Nq;
@@ -637,7 +667,7 @@ __global__ void __launch_bounds__(SKV_THREADS, 1)
   __syncthreads();
   if (warp == SKV_MMA_WARP) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc(tmem, C::TMEM_ALLOC);
   }
 }
 
