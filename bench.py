@@ -26,7 +26,9 @@ bf16 peak, the median SM clock while it ran, its exponential floor and the
 tensor-pipe utilisation from an ncu capture of the same kernel source
 (``profiles/tensor_pipe.txt``, null when the source has changed since).
 ``--profile-grid`` launches every grid point once and nothing else (for that
-ncu capture).
+ncu capture).  The line also carries ``backward`` (fa2_bwd on the headline
+workload) and ``decode`` (the split-K/V entry point on one query against
+16384 keys at d = 128 and against 4096 keys at d = 64), timed the same way.
 
 Decode workloads (``--workload decode_...`` / ``chunk_...``: Nq queries at the
 end of an Nk-long sequence) run the split-K/V entry point instead; a step is
@@ -274,6 +276,90 @@ def run_grid(dev, stream, sampler, peaks, target_ms: float, src: str, sustained_
                               (p["sustained"]["frac_of_sustained_peak"] for p in target if p["sustained"]),
                               default=None)},
     }
+
+
+def burst_time(call, dev, stream, target_ms: float, sampler):
+    """Median per-launch ms of 5 CUDA-event regions of >= 10 back-to-back
+    launches (>= target_ms each) after a 250 ms idle gap; with the median SM
+    clock inside them."""
+    import torch
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    call()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    reps = max(10, int(math.ceil(target_ms / max(ev0.elapsed_time(ev1), 1e-3))))
+    time.sleep(0.25)
+    region_ms, t0 = [], time.time()
+    for _ in range(5):
+        ev0.record(stream)
+        for _ in range(reps):
+            call()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        region_ms.append(ev0.elapsed_time(ev1) / reps)
+    return sorted(region_ms)[2], 5 * reps, sampler.median_between(t0, time.time())
+
+
+DECODE_LINE_WORKLOADS = ("decode_B8_H16_Nk16384_d128", "decode_B32_H16_Nk4096_d64")
+
+
+def decode_lines(dev, stream, sampler, peaks, src, target_ms: float):
+    """The split-K/V entry point on the decode workloads (effective HBM GB/s)."""
+    import torch
+    import exact_tiled_attention_45_b200 as fa2
+    from exact_tiled_attention_45_b200.inputs import WORKLOADS
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    out = {}
+    for name in DECODE_LINE_WORKLOADS:
+        w = WORKLOADS[name]
+        q, k, v = (t.to(dev) for t in workload_inputs(w, 0))
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+        splits = fa2.splitkv_splits(w.B, w.H, w.Nq, w.Nk, w.d, 0)
+        need = fa2.splitkv_workspace_bytes(w.B, w.H, w.Nq, w.Nk, w.d, 0)
+        ws = torch.empty(need, dtype=torch.uint8, device=dev) if need else None
+
+        def call():
+            fa2.fwd_splitkv(q, k, v, causal=w.causal, out=o, lse=lse, workspace=ws, stream=stream)
+
+        ms, launches, mhz = burst_time(call, dev, stream, target_ms, sampler)
+        fa2.sync_status(stream)
+        gbs = w.bytes / (ms * 1e-3) / 1e9
+        out[name] = {"GB_s": round(gbs, 1), "frac_of_copy_bw": round(gbs / hbm, 4), "ms": round(ms, 5),
+                     "n_splits": splits, "launches": launches, "sm_mhz": mhz, "algorithmic_bytes": w.bytes,
+                     "traffic": recorded_traffic(name, src)}
+        del q, k, v, o, lse, ws
+        torch.cuda.empty_cache()
+    return out
+
+
+def backward_line(w, q, k, v, q_host, dev, stream, sampler, peaks, src, target_ms: float):
+    """The backward (fa2_bwd) on the headline workload, TFLOP/s by the 2.5 x
+    forward-FLOP convention."""
+    import torch
+    import exact_tiled_attention_45_b200 as fa2
+    g = torch.Generator(device="cpu")
+    g.manual_seed(1000)
+    do = torch.randn(q_host.shape, generator=g, dtype=torch.float32).to(torch.bfloat16).to(dev)
+    o, lse = fa2.fwd(q, k, v, causal=w.causal, stream=stream)
+    ws = torch.empty(fa2.bwd_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def call():
+        fa2.bwd(q, k, v, o, lse, do, causal=w.causal, dq=dq, dk=dk, dv=dv, workspace=ws, stream=stream)
+
+    ms, launches, mhz = burst_time(call, dev, stream, target_ms, sampler)
+    fa2.sync_status(stream)
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    tf = 2.5 * w.flops / (ms * 1e-3) / 1e12
+    return {"workload": w.name, "tflops": round(tf, 1), "frac": round(tf / peak, 4), "ms": round(ms, 5),
+            "executed_tflops": round((4.0 if w.d > 128 else 3.5) * w.flops / (ms * 1e-3) / 1e12, 1),
+            "launches": launches, "sm_mhz": mhz, "traffic": recorded_traffic(w.name + ":bwd", src),
+            "convention": "2.5 x forward FLOP (five matmuls); the kernels execute seven"}
 
 
 def profile_grid():
@@ -964,9 +1050,15 @@ def main():
 
     peaks, peak_kind = load_peaks()
     src = source_hash()
-    grid = None
+    grid = decode = backward = None
     if not args.no_grid and world == 1:
+        xsampler = ClockSampler(dev)
+        xsampler.start()
+        backward = backward_line(w, q, k, v, q_h, dev, stream, xsampler, peaks, src, args.grid_ms)
         del q, k, v, o, lse
+        torch.cuda.empty_cache()
+        decode = decode_lines(dev, stream, xsampler, peaks, src, args.grid_ms)
+        xsampler.stop()
         torch.cuda.empty_cache()
         gsampler = ClockSampler(dev)
         gsampler.start()
@@ -1032,6 +1124,8 @@ def main():
         "cpu_baseline": cpu,
         "gemm_comparator": gemm,
         "grid": grid,
+        "backward": backward,
+        "decode": decode,
     }
     print(json.dumps(line), flush=True)
     return 0
