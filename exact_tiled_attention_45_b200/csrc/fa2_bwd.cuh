@@ -154,15 +154,41 @@ __device__ __forceinline__ void bwd_item(const BwdParams& p, int& bh, int& tile)
   tile = (CAUSAL && HEAVY_IS_LAST) ? (p.n_tiles - 1 - rank) : rank;
 }
 
-// Row-major bf16 row store of 32 fp32 accumulator columns (times f).
-__device__ __forceinline__ void store_row32_bf16(__nv_bfloat16* dst, const uint32_t (&a)[32], float f) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
+// Row r of an NC-column fp32 accumulator in TMEM, times f, as bf16 into a
+// 128-row tile in shared memory laid out for TMA stores of 64-column boxes
+// with 128-byte swizzle: 64-column chunk c at tile + c * 16 KB, row r at
+// r * 128 bytes, 16-byte unit k of the row at (k ^ (r mod 8)) * 16.  Up to
+// 128 columns are loaded from TMEM at a time.
+template <int NC>
+__device__ __forceinline__ void stage_row_bf16(uint32_t tile, uint32_t taddr, int r, float f) {
+  constexpr int G = (NC < 128 ? NC : 128) / 32;
+  const uint64_t ff = f2_pack(f, f);
 #pragma unroll
-  for (int e = 0; e < 32; e += 8)
-    d4[e / 8] = make_uint4(pack_bf16x2(__uint_as_float(a[e]) * f, __uint_as_float(a[e + 1]) * f),
-                           pack_bf16x2(__uint_as_float(a[e + 2]) * f, __uint_as_float(a[e + 3]) * f),
-                           pack_bf16x2(__uint_as_float(a[e + 4]) * f, __uint_as_float(a[e + 5]) * f),
-                           pack_bf16x2(__uint_as_float(a[e + 6]) * f, __uint_as_float(a[e + 7]) * f));
+  for (int g = 0; g < NC / 32; g += G) {
+    uint32_t a[G][32];
+#pragma unroll
+    for (int cc = 0; cc < G; ++cc) tmem_ld32(taddr + (g + cc) * 32, a[cc]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int cc = 0; cc < G; ++cc) reg_fence32(a[cc]);
+#pragma unroll
+    for (int cc = 0; cc < G; ++cc) {
+      const int c32 = g + cc;
+      uint32_t w[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        float x0, x1;
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(a[cc][2 * e]), __uint_as_float(a[cc][2 * e + 1])), ff), x0, x1);
+        w[e] = pack_bf16x2(x0, x1);
+      }
+      const uint32_t line = tile + static_cast<uint32_t>(c32 >> 1) * (128u * 128u) + static_cast<uint32_t>(r) * 128u;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int k = (c32 & 1) * 4 + v;
+        st_shared_v4(line + ((k ^ (r & 7)) << 4), w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+      }
+    }
+  }
 }
 
 // dS for NC keys (or queries) of one row: reads dP from TMEM 32 columns at a
@@ -195,6 +221,7 @@ struct DqBars {
   uint64_t k_full[4], k_empty[4];
   uint64_t v_full[4], v_empty[4];
   uint64_t s_full, s_free, dp_full, ds_ready, mma_final;
+  uint64_t epi;  // the four elementwise warps staged their gradient rows in shared memory
   uint32_t tmem_base;
   int abort;
 };
@@ -207,7 +234,7 @@ template <int HD, bool CAUSAL>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                      const BwdParams p) {
+                      const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using C = BwdCfg<HD>;
   constexpr int BNK = C::BNK;
   int bh, qt;
@@ -242,6 +269,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     mbar_init(smem_u32(&bars->dp_full), 1);
     mbar_init(smem_u32(&bars->ds_ready), 4);
     mbar_init(smem_u32(&bars->mma_final), 1);
+    mbar_init(smem_u32(&bars->epi), 4);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -424,23 +452,21 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     }
     if (ok) ok = wait_warp(smem_u32(&bars->mma_final), 0, abort_flag, to);
     if (ok) {
+      // Every MMA has completed, so the Q tile's buffer takes dQ (bf16, times
+      // the softmax scale) for one TMA store per 64 columns; the store skips
+      // rows past N and columns past d.  Only the storing thread waits
+      // (bounded) for the four warps, so a warp that gave up earlier cannot
+      // leave the others blocked.
       tc_fence_after();
-      __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bh) * p.N + row) * p.d;
-      // Up to 128 columns at a time (256 registers of dQ would not fit).
-      constexpr int GROUP = (HD < 128 ? HD : 128) / 32;
+      stage_row_bf16<HD>(sQ, lane_addr + BQ_DQ, r, p.scale);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->epi));
+      if (threadIdx.x == 0 && wait_bounded(smem_u32(&bars->epi), 0, abort_flag, to, ROLE_SOFTMAX)) {
 #pragma unroll
-      for (int g = 0; g < HD / 32; g += GROUP) {
-        uint32_t a[GROUP][32];
-#pragma unroll
-        for (int cc = 0; cc < GROUP; ++cc) tmem_ld32(lane_addr + BQ_DQ + (g + cc) * 32, a[cc]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int cc = 0; cc < GROUP; ++cc) reg_fence32(a[cc]);
-        if (valid) {
-#pragma unroll
-          for (int cc = 0; cc < GROUP; ++cc)
-            if ((g + cc) * 32 < p.d) store_row32_bf16(dst + (g + cc) * 32, a[cc], p.scale);
-        }
+        for (int cc = 0; cc < HD / 64; ++cc) tma_store_3d(&tm_dq, sQ + cc * C::CHUNK_BYTES, cc * 64, q0, bh);
+        bulk_commit_group();
+        bulk_wait_read();  // the shared-memory source must stay valid until read
       }
     }
   }
@@ -457,6 +483,7 @@ struct KvBars {
   uint64_t kv_full;
   uint64_t q_full[3], q_empty[3];
   uint64_t s_full, dp_full, p_ready, ds_ready, mma_final;
+  uint64_t epi;  // the four elementwise warps staged their gradient rows in shared memory
   uint32_t tmem_base;
   int abort;
 };
@@ -471,6 +498,7 @@ template <int HD, bool CAUSAL, int PASS>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                        const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                         const BwdParams p) {
   using C = BwdCfg<HD>;
   constexpr int BMQ = C::BMQ;
@@ -506,6 +534,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     mbar_init(smem_u32(&bars->p_ready), 4);
     mbar_init(smem_u32(&bars->ds_ready), 4);
     mbar_init(smem_u32(&bars->mma_final), 1);
+    mbar_init(smem_u32(&bars->epi), 4);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -692,28 +721,24 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     }
     if (ok) ok = wait_warp(smem_u32(&bars->mma_final), 0, abort_flag, to);
     if (ok) {
+      // Every MMA has completed: the V tile's buffer takes dV and the K
+      // tile's dK (bf16; dK times the softmax scale) for TMA stores of 64
+      // columns each, which skip rows past N and columns past d.  Only the
+      // storing thread waits (bounded) for the four warps.
       tc_fence_after();
-      const bool valid = key < p.N;
-      const size_t off = (static_cast<size_t>(bh) * p.N + key) * p.d;
-      if constexpr (DO_DV) {
+      if constexpr (DO_DV) stage_row_bf16<HD>(sV, lane_addr + BK_DV, r, 1.f);
+      if constexpr (DO_DK) stage_row_bf16<HD>(sK, lane_addr + BK_DK, r, p.scale);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->epi));
+      if (threadIdx.x == 0 && wait_bounded(smem_u32(&bars->epi), 0, abort_flag, to, ROLE_SOFTMAX)) {
 #pragma unroll
-        for (int cc = 0; cc < HD / 32; ++cc) {
-          uint32_t a[32];
-          tmem_ld32(lane_addr + BK_DV + cc * 32, a);
-          tmem_wait_ld();
-          reg_fence32(a);
-          if (valid && cc * 32 < p.d) store_row32_bf16(p.dv + off + cc * 32, a, 1.f);
+        for (int cc = 0; cc < HD / 64; ++cc) {
+          if constexpr (DO_DV) tma_store_3d(&tm_dv, sV + cc * C::CHUNK_BYTES, cc * 64, k0, bh);
+          if constexpr (DO_DK) tma_store_3d(&tm_dk, sK + cc * C::CHUNK_BYTES, cc * 64, k0, bh);
         }
-      }
-      if constexpr (DO_DK) {
-#pragma unroll
-        for (int cc = 0; cc < HD / 32; ++cc) {
-          uint32_t a[32];
-          tmem_ld32(lane_addr + BK_DK + cc * 32, a);
-          tmem_wait_ld();
-          reg_fence32(a);
-          if (valid && cc * 32 < p.d) store_row32_bf16(p.dk + off + cc * 32, a, p.scale);
-        }
+        bulk_commit_group();
+        bulk_wait_read();  // the shared-memory sources must stay valid until read
       }
     }
   }

@@ -1044,6 +1044,7 @@ static int bwd_set_smem(Kern kern, int bytes) {
 struct BwdMaps {
   CUtensorMap q128, do128, k_dq, v_dq;  // dQ kernel
   CUtensorMap k128, v128, q_kv, do_kv;  // dK/dV kernel(s)
+  CUtensorMap dq128, dk128, dv128;       // gradient stores (128-row boxes)
 };
 
 template <int HD, bool CAUSAL>
@@ -1067,21 +1068,21 @@ static int bwd_launch_t(const BwdMaps& m, const BwdParams& prm, cudaStream_t str
     if (dev < 32) attr_done_mask.fetch_or(1u << dev, std::memory_order_acq_rel);
   }
   const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_tiles);
-  kq<<<grid, BWD_THREADS, C::DQ_SMEM, stream>>>(m.q128, m.k_dq, m.v_dq, m.do128, prm);
+  kq<<<grid, BWD_THREADS, C::DQ_SMEM, stream>>>(m.q128, m.k_dq, m.v_dq, m.do128, m.dq128, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_detail("dQ kernel launch: %s", cudaGetErrorString(e));
     return FA2_ERR_CUDA;
   }
-  kkv<<<grid, BWD_THREADS, C::KV_SMEM, stream>>>(m.q_kv, m.k128, m.v128, m.do_kv, prm);
+  kkv<<<grid, BWD_THREADS, C::KV_SMEM, stream>>>(m.q_kv, m.k128, m.v128, m.do_kv, m.dk128, m.dv128, prm);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_detail("dK/dV kernel launch: %s", cudaGetErrorString(e));
     return FA2_ERR_CUDA;
   }
   if constexpr (HD == 256) {
-    fa2_bwd_dkdv_kernel<HD, CAUSAL, BWD_KV_DK><<<grid, BWD_THREADS, C::KV_SMEM, stream>>>(m.q_kv, m.k128, m.v128,
-                                                                                         m.do_kv, prm);
+    fa2_bwd_dkdv_kernel<HD, CAUSAL, BWD_KV_DK><<<grid, BWD_THREADS, C::KV_SMEM, stream>>>(
+        m.q_kv, m.k128, m.v128, m.do_kv, m.dk128, m.dv128, prm);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
       set_detail("dK kernel launch: %s", cudaGetErrorString(e));
@@ -1157,6 +1158,9 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   if ((st = make_tmap(&maps.v_dq, v, d, N, bhi, tile_small)) != FA2_OK) return st;
   if ((st = make_tmap(&maps.q_kv, q, d, N, bhi, tile_small)) != FA2_OK) return st;
   if ((st = make_tmap(&maps.do_kv, dout, d, N, bhi, tile_small)) != FA2_OK) return st;
+  if ((st = make_tmap(&maps.dq128, dq, d, N, bhi)) != FA2_OK) return st;
+  if ((st = make_tmap(&maps.dk128, dk, d, N, bhi)) != FA2_OK) return st;
+  if ((st = make_tmap(&maps.dv128, dv, d, N, bhi)) != FA2_OK) return st;
   BwdParams prm;
   prm.o = static_cast<const __nv_bfloat16*>(o);
   prm.dout = static_cast<const __nv_bfloat16*>(dout);
