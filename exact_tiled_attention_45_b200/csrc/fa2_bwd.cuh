@@ -396,23 +396,47 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     // D = dO . O and -LSE*log2(e) of this row, kept in registers and written
     // to the workspace for the dK/dV kernel (padding rows: D = 0, -inf).
-    float dsum = 0.f, nlse2 = -INFINITY;
-    if (valid) {
-      const size_t off = (static_cast<size_t>(bh) * p.N + row) * p.d;
-      const uint4* o4 = reinterpret_cast<const uint4*>(p.o + off);
-      const uint4* g4 = reinterpret_cast<const uint4*>(p.dout + off);
-#pragma unroll 4
-      for (int c = 0; c < p.d / 8; ++c) {
-        const uint4 a = o4[c], g = g4[c];
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
+    // O and dO are read row-coalesced: LPR lanes cover one row, 16 bytes
+    // each, RPI rows per load instruction; the row's partial dot products
+    // are summed across its lanes and handed to the thread that owns it.
+    float dsum = 0.f;
+    {
+      constexpr int NV = HD / 8;              // 16-byte vectors per row
+      constexpr int LPR = NV < 32 ? NV : 32;  // lanes per row
+      constexpr int RPI = 32 / LPR;           // rows per load instruction
+      constexpr int NI = 32 / RPI;            // load instructions per warp
+      constexpr int BATCH = NI < 8 ? NI : 8;
+      const int sub = lane % LPR, grp = lane / LPR;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          dsum = fmaf(__uint_as_float(aw[e] << 16), __uint_as_float(gw[e] << 16), dsum);
-          dsum = fmaf(__uint_as_float(aw[e] & 0xffff0000u), __uint_as_float(gw[e] & 0xffff0000u), dsum);
+      for (int b0 = 0; b0 < NI; b0 += BATCH) {
+        uint4 a[BATCH], g[BATCH];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+          const int rw = q0 + warp * 32 + (b0 + i) * RPI + grp;
+          a[i] = g[i] = make_uint4(0u, 0u, 0u, 0u);
+          if (rw < p.N && sub * 8 < p.d) {  // columns past d (padded head dimension) are not read
+            const size_t off = (static_cast<size_t>(bh) * p.N + rw) * p.d + sub * 8;
+            a[i] = *reinterpret_cast<const uint4*>(p.o + off);
+            g[i] = *reinterpret_cast<const uint4*>(p.dout + off);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+          const uint32_t aw[4] = {a[i].x, a[i].y, a[i].z, a[i].w}, gw[4] = {g[i].x, g[i].y, g[i].z, g[i].w};
+          float part = 0.f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            part = fmaf(__uint_as_float(aw[e] << 16), __uint_as_float(gw[e] << 16), part);
+            part = fmaf(__uint_as_float(aw[e] & 0xffff0000u), __uint_as_float(gw[e] & 0xffff0000u), part);
+          }
+#pragma unroll
+          for (int m = LPR / 2; m > 0; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
+          const float row_sum = __shfl_sync(0xffffffffu, part, (lane % RPI) * LPR);
+          if (lane / RPI == b0 + i) dsum = row_sum;
         }
       }
-      nlse2 = -p.lse[static_cast<size_t>(bh) * p.N + row] * LOG2E_F;
     }
+    const float nlse2 = valid ? -p.lse[static_cast<size_t>(bh) * p.N + row] * LOG2E_F : -INFINITY;
     const size_t vrow = static_cast<size_t>(bh) * p.n_tiles * BM + q0 + r;
     p.dvec[vrow] = dsum;
     p.lse2[vrow] = nlse2;
