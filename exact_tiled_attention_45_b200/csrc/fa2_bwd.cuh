@@ -217,7 +217,7 @@ __device__ __forceinline__ void ds_to_tmem(uint32_t dp_addr, const float (&p)[NC
 }
 
 struct DqBars {
-  uint64_t qdo_full;
+  uint64_t q_full, do_full;  // the resident Q and dO tiles (S waits for Q only)
   uint64_t k_full[4], k_empty[4];
   uint64_t v_full[4], v_empty[4];
   uint64_t s_full, s_free, dp_full, ds_ready, mma_final;
@@ -255,7 +255,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   const uint32_t sK = base + C::DQ_OFF_K, sV = base + C::DQ_OFF_V;
 
   if (threadIdx.x == 0) {
-    mbar_init(smem_u32(&bars->qdo_full), 1);
+    mbar_init(smem_u32(&bars->q_full), 1);
+    mbar_init(smem_u32(&bars->do_full), 1);
     for (int s = 0; s < C::DQ_KS; ++s) {
       mbar_init(smem_u32(&bars->k_full[s]), 1);
       mbar_init(smem_u32(&bars->k_empty[s]), 1);
@@ -291,14 +292,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 
   if (warp == BWD_PRODUCER_WARP) {
     if (lane == 0) {
-      const uint32_t bq = smem_u32(&bars->qdo_full);
+      // Q, K(0), dO, V(0): the order the first two MMAs need them.
+      const uint32_t bq = smem_u32(&bars->q_full), bdo = smem_u32(&bars->do_full);
       const bool load_qdo = p.inject_timeout != 1;
       if (load_qdo) {
-        mbar_arrive_expect_tx(bq, 2 * C::TILE_BYTES);
-        for (int c = 0; c < C::KCH; ++c) {
-          tma_load_3d(sQ + c * C::CHUNK_BYTES, &tm_q, bq, c * 64, q0, bh);
-          tma_load_3d(sDO + c * C::CHUNK_BYTES, &tm_do, bq, c * 64, q0, bh);
-        }
+        mbar_arrive_expect_tx(bq, C::TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c) tma_load_3d(sQ + c * C::CHUNK_BYTES, &tm_q, bq, c * 64, q0, bh);
       }
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < nkv; ++j) {
@@ -311,6 +310,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         for (int c = 0; c < C::KCH; ++c)
           tma_load_3d(sK + ks * C::KV_TILE + c * C::KV_CHUNK, &tm_k, kb, c * 64, j * BNK, bh);
         ++k_issued;
+        if (j == 0 && load_qdo) {
+          mbar_arrive_expect_tx(bdo, C::TILE_BYTES);
+          for (int c = 0; c < C::KCH; ++c) tma_load_3d(sDO + c * C::CHUNK_BYTES, &tm_do, bdo, c * 64, q0, bh);
+        }
         if (j >= C::DQ_VS &&
             !wait_bounded(smem_u32(&bars->v_empty[vs]), ((j / C::DQ_VS) - 1) & 1, abort_flag, to, ROLE_PRODUCER))
           break;
@@ -320,7 +323,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           tma_load_3d(sV + vs * C::KV_TILE + c * C::KV_CHUNK, &tm_v, vb, c * 64, j * BNK, bh);
         ++v_issued;
       }
-      if (load_qdo) wait_drain(bq, 0, to);
+      if (load_qdo) {
+        wait_drain(bq, 0, to);
+        if (k_issued > 0) wait_drain(bdo, 0, to);
+      }
       for (int x = (k_issued > C::DQ_KS ? k_issued - C::DQ_KS : 0); x < k_issued; ++x)
         wait_drain(smem_u32(&bars->k_full[x % C::DQ_KS]), (x / C::DQ_KS) & 1, to);
       for (int x = (v_issued > C::DQ_VS ? v_issued - C::DQ_VS : 0); x < v_issued; ++x)
@@ -341,13 +347,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                  smem_desc_sw128(b + (kk >> 2) * C::KV_CHUNK + in_chunk, 16, 1024), IDESC_SS, kk > 0 ? 1u : 0u);
         }
       };
-      bool ok = wait_bounded(smem_u32(&bars->qdo_full), 0, abort_flag, to, ROLE_MMA);
+      bool ok = wait_bounded(smem_u32(&bars->q_full), 0, abort_flag, to, ROLE_MMA);
       ok = ok && wait_bounded(smem_u32(&bars->k_full[0]), 0, abort_flag, to, ROLE_MMA);
       if (ok) {
         tc_fence_after();
         mma_kmajor(tmem + BQ_S, sQ, sK);
         mma_commit(smem_u32(&bars->s_full));
       }
+      ok = ok && wait_bounded(smem_u32(&bars->do_full), 0, abort_flag, to, ROLE_MMA);
       ok = ok && wait_bounded(smem_u32(&bars->v_full[0]), 0, abort_flag, to, ROLE_MMA);
       if (ok) {
         tc_fence_after();
@@ -504,7 +511,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 }
 
 struct KvBars {
-  uint64_t kv_full;
+  uint64_t k_full, v_full;  // the resident K and V tiles (S^T waits for K only)
   uint64_t q_full[3], q_empty[3];
   uint64_t s_full, dp_full, p_ready, ds_ready, mma_final;
   uint64_t epi;  // the four elementwise warps staged their gradient rows in shared memory
@@ -548,7 +555,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   const float* vec = reinterpret_cast<const float*>(smem + C::KV_OFF_VEC);
 
   if (threadIdx.x == 0) {
-    mbar_init(smem_u32(&bars->kv_full), 1);
+    mbar_init(smem_u32(&bars->k_full), 1);
+    mbar_init(smem_u32(&bars->v_full), 1);
     for (int s = 0; s < C::KV_QS; ++s) {
       mbar_init(smem_u32(&bars->q_full[s]), 1);
       mbar_init(smem_u32(&bars->q_empty[s]), 1);
@@ -581,14 +589,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 
   if (warp == BWD_PRODUCER_WARP) {
     if (lane == 0) {
-      const uint32_t bkv = smem_u32(&bars->kv_full);
+      // K, then the first (Q, dO, lse2, D) stage, then V (read by dP^T
+      // only; the dV pass of d = 256 does not read it).
+      const uint32_t bk = smem_u32(&bars->k_full), bv = smem_u32(&bars->v_full);
       const bool load_kv = p.inject_timeout != 2;
       if (load_kv) {
-        mbar_arrive_expect_tx(bkv, 2 * C::TILE_BYTES);
-        for (int c = 0; c < C::KCH; ++c) {
-          tma_load_3d(sK + c * C::CHUNK_BYTES, &tm_k, bkv, c * 64, k0, bh);
-          tma_load_3d(sV + c * C::CHUNK_BYTES, &tm_v, bkv, c * 64, k0, bh);
-        }
+        mbar_arrive_expect_tx(bk, C::TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c) tma_load_3d(sK + c * C::CHUNK_BYTES, &tm_k, bk, c * 64, k0, bh);
       }
       int issued = 0;
       for (int t = 0; t < nq; ++t) {
@@ -606,9 +613,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         const uint32_t sv = base + C::KV_OFF_VEC + s * 1024;
         bulk_load_1d(sv, p.lse2 + vec_head + i * BMQ, BMQ * 4, bq);
         bulk_load_1d(sv + 512, p.dvec + vec_head + i * BMQ, BMQ * 4, bq);
+        if (DO_DK && t == 0 && load_kv) {
+          mbar_arrive_expect_tx(bv, C::TILE_BYTES);
+          for (int c = 0; c < C::KCH; ++c) tma_load_3d(sV + c * C::CHUNK_BYTES, &tm_v, bv, c * 64, k0, bh);
+        }
         ++issued;
       }
-      if (load_kv) wait_drain(bkv, 0, to);
+      if (load_kv) {
+        wait_drain(bk, 0, to);
+        if (DO_DK && issued > 0) wait_drain(bv, 0, to);
+      }
       for (int x = (issued > C::KV_QS ? issued - C::KV_QS : 0); x < issued; ++x)
         wait_drain(smem_u32(&bars->q_full[x % C::KV_QS]), (x / C::KV_QS) & 1, to);
     }
@@ -636,13 +650,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b + kk * 2048, C::Q_CHUNK, 1024), IDESC_ACC,
                  (acc || kk > 0) ? 1u : 0u);
       };
-      bool ok = wait_bounded(smem_u32(&bars->kv_full), 0, abort_flag, to, ROLE_MMA) &&
+      bool ok = wait_bounded(smem_u32(&bars->k_full), 0, abort_flag, to, ROLE_MMA) &&
                 wait_bounded(smem_u32(&bars->q_full[0]), 0, abort_flag, to, ROLE_MMA);
       if (ok) {
         tc_fence_after();
         mma_kmajor(tmem + BK_S, sK, sQ);
         mma_commit(smem_u32(&bars->s_full));
-        if constexpr (DO_DK) {
+      }
+      if constexpr (DO_DK) {
+        ok = ok && wait_bounded(smem_u32(&bars->v_full), 0, abort_flag, to, ROLE_MMA);
+        if (ok) {
+          tc_fence_after();
           mma_kmajor(tmem + BK_DP, sV, sDO);
           mma_commit(smem_u32(&bars->dp_full));
         }

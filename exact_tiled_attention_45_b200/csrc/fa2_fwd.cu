@@ -457,17 +457,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (warp == PRODUCER_WARP && lane == 0) {
       // ---------------------------------------------------------- TMA producer
       const bool load_q = !p.inject_timeout;
-      if (load_q) {
-        for (int t = 0; t < 2; ++t) {
-          // A tile that starts at or past N has no row to store; it is loaded
-          // from tile 0's rows so that no copy lies wholly outside the tensor.
-          const int qy = (q0 + t * BM < p.N) ? q0 + t * BM : q0;
-          const uint32_t qbar = smem_u32(&bars->q_full[t]);
-          mbar_arrive_expect_tx(qbar, C::TILE_BYTES);
-          for (int c = 0; c < C::KCH; ++c)
-            tma_load_3d(sQ + t * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, qbar, c * 64, qy, bh);
-        }
-      }
+      // Q_0, K_0, Q_1, V_0, then K and V: the order the first MMAs need them.
+      auto load_q_tile = [&](int t) {
+        // A tile that starts at or past N has no row to store; it is loaded
+        // from tile 0's rows so that no copy lies wholly outside the tensor.
+        const int qy = (q0 + t * BM < p.N) ? q0 + t * BM : q0;
+        const uint32_t qbar = smem_u32(&bars->q_full[t]);
+        mbar_arrive_expect_tx(qbar, C::TILE_BYTES);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_3d(sQ + t * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, qbar, c * 64, qy, bh);
+      };
+      if (load_q) load_q_tile(0);
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < n1; ++j) {
         const int ks = j % C::KS;
@@ -481,6 +481,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int c = 0; c < C::KCH; ++c)
           tma_load_3d(sK + ks * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_k, kb, c * 64, j * BN, bh);
         ++k_issued;
+        if (j == 0 && load_q) load_q_tile(1);
         const int vs = j % C::VS;
         if (j >= C::VS &&
             !wait_bounded(smem_u32(&bars->v_empty[vs]), ((j / C::VS) - 1) & 1, abort_flag, p.timeout_ns,
