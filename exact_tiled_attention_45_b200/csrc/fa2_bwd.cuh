@@ -403,33 +403,44 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     // D = dO . O and -LSE*log2(e) of this row, kept in registers and written
     // to the workspace for the dK/dV kernel (padding rows: D = 0, -inf).
-    // O and dO are read row-coalesced: LPR lanes cover one row, 16 bytes
-    // each, RPI rows per load instruction; the row's partial dot products
-    // are summed across its lanes and handed to the thread that owns it.
+    // O is read row-coalesced from global memory (LPR lanes per row, 16
+    // bytes each, RPI rows per load instruction, up to 16 loads of a lane in
+    // flight); dO too at d = 64, and from the resident tile in shared memory
+    // once its load has landed at d >= 128 (measured: the global loads win
+    // at d = 64, the shared tile at d = 128).  Each row's partial dot
+    // products are summed across its lanes and handed to the row's thread.
+    bool ok = true;
     float dsum = 0.f;
     {
       constexpr int NV = HD / 8;              // 16-byte vectors per row
       constexpr int LPR = NV < 32 ? NV : 32;  // lanes per row
       constexpr int RPI = 32 / LPR;           // rows per load instruction
       constexpr int NI = 32 / RPI;            // load instructions per warp
-      constexpr int BATCH = NI < 8 ? NI : 8;
+      constexpr int BATCH = NI < 16 ? NI : 16;
       const int sub = lane % LPR, grp = lane / LPR;
+      const uint32_t unit = static_cast<uint32_t>(sub >> 3) * C::CHUNK_BYTES;  // 64-column chunk of this lane's 16 bytes
 #pragma unroll
-      for (int b0 = 0; b0 < NI; b0 += BATCH) {
-        uint4 a[BATCH], g[BATCH];
+      for (int b0 = 0; b0 < NI && ok; b0 += BATCH) {
+        uint4 a[BATCH], gg[BATCH];
 #pragma unroll
         for (int i = 0; i < BATCH; ++i) {
           const int rw = q0 + warp * 32 + (b0 + i) * RPI + grp;
-          a[i] = g[i] = make_uint4(0u, 0u, 0u, 0u);
+          a[i] = gg[i] = make_uint4(0u, 0u, 0u, 0u);
           if (rw < p.N && sub * 8 < p.d) {  // columns past d (padded head dimension) are not read
             const size_t off = (static_cast<size_t>(bh) * p.N + rw) * p.d + sub * 8;
             a[i] = *reinterpret_cast<const uint4*>(p.o + off);
-            g[i] = *reinterpret_cast<const uint4*>(p.dout + off);
+            if constexpr (HD == 64) gg[i] = *reinterpret_cast<const uint4*>(p.dout + off);
           }
         }
+        if (HD > 64 && b0 == 0) ok = wait_warp(smem_u32(&bars->do_full), 0, abort_flag, to);
+        if (!ok) break;
 #pragma unroll
         for (int i = 0; i < BATCH; ++i) {
-          const uint32_t aw[4] = {a[i].x, a[i].y, a[i].z, a[i].w}, gw[4] = {g[i].x, g[i].y, g[i].z, g[i].w};
+          // the tile's dO row (zero past N and past d), 128-byte swizzle
+          const int rt = warp * 32 + (b0 + i) * RPI + grp;
+          const uint4 g =
+              (HD == 64) ? gg[i] : ld_shared_v4(sDO + unit + rt * 128 + (((sub & 7) ^ (rt & 7)) << 4));
+          const uint32_t aw[4] = {a[i].x, a[i].y, a[i].z, a[i].w}, gw[4] = {g.x, g.y, g.z, g.w};
           float part = 0.f;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -444,13 +455,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       }
     }
     const float nlse2 = valid ? -p.lse[static_cast<size_t>(bh) * p.N + row] * LOG2E_F : -INFINITY;
-    const size_t vrow = static_cast<size_t>(bh) * p.n_tiles * BM + q0 + r;
-    p.dvec[vrow] = dsum;
-    p.lse2[vrow] = nlse2;
+    if (ok) {
+      const size_t vrow = static_cast<size_t>(bh) * p.n_tiles * BM + q0 + r;
+      p.dvec[vrow] = dsum;
+      p.lse2[vrow] = nlse2;
+    }
 
     const float c = p.scale_log2;
-    bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
+    for (int j = 0; ok && j < nkv; ++j) {
       ok = wait_warp(smem_u32(&bars->s_full), j & 1, abort_flag, to);
       if (!ok) break;
       tc_fence_after();
