@@ -43,14 +43,19 @@ constexpr float LOG2E_F = 1.4426950408889634f;
 // Of every 8 pairs of exponentials 2^(c*s - LSE*log2(e)), this many run on
 // the FMA-pipe polynomial (exp2_poly_pair) and the rest on the
 // special-function unit; the arguments are <= 0 (P <= 1), -inf when masked.
-#ifndef FA2_BWD_EMU_PAIRS
-#define FA2_BWD_EMU_PAIRS 2
+// Measured: 1 of 8 is fastest at d = 128 (+1.1 % over 2 at the headline
+// shape), 2 of 8 at d = 64 (where the MMAs per exponential are half).
+#ifndef FA2_BWD_EMU_PAIRS_D64
+#define FA2_BWD_EMU_PAIRS_D64 2
+#endif
+#ifndef FA2_BWD_EMU_PAIRS_WIDE
+#define FA2_BWD_EMU_PAIRS_WIDE 1  // d = 128 and 256
 #endif
 
 // P of NC keys (or queries) of one row: pr[e] = 2^(c * s[e] + nl[e]), where
 // nl is -LSE*log2(e) (one value per row, or per column when `per_col`);
 // masked entries (e past `lim` on a masked tile, see the callers) give 0.
-template <bool PER_COL, int NC>
+template <bool PER_COL, int NC, int EMU>
 __device__ __forceinline__ void bwd_probs(float (&pr)[NC], const uint32_t (&s)[NC], float c, float nl_row,
                                           const float* nl_col, bool masked, int lim, bool mask_below) {
   const uint64_t cc = f2_pack(c, c);
@@ -66,7 +71,7 @@ __device__ __forceinline__ void bwd_probs(float (&pr)[NC], const uint32_t (&s)[N
     uint64_t nl = nlr;
     if (PER_COL) nl = *reinterpret_cast<const uint64_t*>(nl_col + e);
     const uint64_t x = f2_fma(f2_pack(x0, x1), cc, nl);
-    if (((e >> 1) & 7) < FA2_BWD_EMU_PAIRS) {
+    if (((e >> 1) & 7) < EMU) {
       f2_unpack(exp2_poly_pair(x), pr[e], pr[e + 1]);
     } else {
       float a0, a1;
@@ -81,6 +86,7 @@ template <int HD>
 struct BwdCfg {
   static_assert(HD == 64 || HD == 128 || HD == 256, "head dimension");
   static constexpr int KCH = HD / 64;
+  static constexpr int EMU_PAIRS = (HD == 64) ? FA2_BWD_EMU_PAIRS_D64 : FA2_BWD_EMU_PAIRS_WIDE;
   static constexpr int CHUNK_BYTES = 128 * 128;          // 128 rows x 128 bytes
   static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;   // one 128-row tile
   // dQ kernel: Q and dO resident, K and V rings of BNK-key tiles.
@@ -482,7 +488,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         const bool diag = CAUSAL && (kv0 + BNK - 1 > q0);  // the tile reaches past the first row
         const bool tail = !CAUSAL && (kv0 + BNK > p.N);
         const int lim = diag ? (row - kv0) : (p.N - 1 - kv0);  // last allowed key column
-        bwd_probs<false, BNK>(pr, s, c, nlse2, nullptr, diag || tail, lim, false);
+        bwd_probs<false, BNK, C::EMU_PAIRS>(pr, s, c, nlse2, nullptr, diag || tail, lim, false);
       }
       ok = wait_warp(smem_u32(&bars->dp_full), j & 1, abort_flag, to);
       if (!ok) break;
@@ -746,7 +752,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         // Query i*BMQ + e sees this key only if i*BMQ + e >= key.
         const int q_first = i * BMQ;
         const bool diag = CAUSAL && (q_first < k0 + BN - 1);
-        bwd_probs<true, BMQ>(pr, sv, c, 0.f, l2, diag, key - q_first, true);
+        bwd_probs<true, BMQ, C::EMU_PAIRS>(pr, sv, c, 0.f, l2, diag, key - q_first, true);
       }
       if constexpr (DO_DV) {
         // P^T (bf16) over the first BMQ/2 score columns, for dV += P^T dO.
