@@ -47,3 +47,16 @@ def test_tensor_pipe_record_is_keyed_by_source(tmp_path, monkeypatch):
     assert rec == {"grid_N512_d64_full": {"tensor_pipe_pct": 41.5, "tensor_pipe_active_pct": 44.0,
                                           "traffic": 2.7e8}}
     assert bench.recorded_tensor_pipe("zzz") == {}
+
+
+def test_source_hash_covers_every_kernel_source():
+    # The ncu records in profiles/ are trusted only while this hash matches,
+    # so every file the library is compiled from must be part of it, and
+    # the rebuild check must watch the same files.
+    import glob
+    from exact_tiled_attention_45_b200 import build
+    csrc = os.path.join(bench.ROOT, "exact_tiled_attention_45_b200", "csrc")
+    kernel_files = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")))
+    hashed = sorted(os.path.join(bench.ROOT, rel) for rel in bench.KERNEL_SOURCES)
+    assert kernel_files == hashed
+    assert set(kernel_files) <= {os.path.abspath(p) for p in build.DEPS}
